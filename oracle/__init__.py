@@ -1,0 +1,17 @@
+"""The CPU oracle for the NVFP4 MoE FFN layer.
+
+TEST INFRASTRUCTURE.  This package is a plain, slow, fp64 restatement of what
+the layer computes, written before and independently of the CUDA path: it
+shares no code, headers, tables or helpers with ``moe_expert_layer_renorm_b200``
+and never imports it (and vice versa).  Only ``tests/``, ``__graft_entry__.smoke()``
+and ``bench.py``'s CPU-baseline leg may import it.
+
+Modules:
+  nvfp4      - E2M1/E4M3 decode from bits, NVFP4 decode and pack
+  moe_layer  - route, permute, SwiGLU expert FFN, combine, tolerance
+
+Every function is pinned by a ``-m "not gpu"`` test against something other
+than itself (hand-worked tables, closed forms, brute force, a library routine
+for a special case); nothing is "parity unpinned".
+"""
+from . import nvfp4, moe_layer  # noqa: F401
