@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of one NVFP4 MoE FFN layer on B200 through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole layer (route -> permute -> gate/up GEMM +
+SwiGLU -> down GEMM -> combine) over one batch of synthetic tokens.  Steps
+rotate over R independent layers (own weights, activations and logits) so
+that the expert weights a step reads are not in L2 from the step before.
+Prints one JSON line on rank 0.  With N > 1 (torchrun) every rank runs its
+own independent batches (weak scaling; no data-path collective) and the time
+is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_expert_layer_renorm_b200 import inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOP/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_T64", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=4, help="independent layers the steps rotate over")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample-tokens", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def bytes_per_expert(H: int, I: int) -> int:
+    """Algorithmic NVFP4 bytes of one expert: codes + unpadded scales + 3 fp32 globals."""
+    return 3 * (H * I // 2 + H * I // 16) + 12
+
+
+def gate_up_bytes_per_expert(H: int, I: int) -> int:
+    return 2 * (H * I // 2 + H * I // 16) + 8
+
+
+# ---------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.idx), "-lms", "200"], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.out.read())) if len(r) >= 9]
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ our arm ---
+
+def traffic_record(kernel_src: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(key)
+    if not rec:
+        return None
+    with open(kernel_src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if rec.get("src_sha256_16") == h else None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from moe_expert_layer_renorm_b200 import _lib
+    from moe_expert_layer_renorm_b200.layer import ExpertPool, MoELayer
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = inputs.WORKLOADS[args.workload]
+    R = max(1, args.layers)
+    T = w.T
+    # per-rank, per-layer independent inputs
+    layers = []
+    for l in range(R):
+        s = inputs.layer_seed(w.seed + 1_000_003 * rank, l)
+        li = inputs.make_layer_inputs(inputs.custom_workload(w, seed=s), 0)
+        st = li.slot_table
+        pool = ExpertPool(w.H, w.I, w.slots, device=dev)
+        for e in range(w.E):
+            for mat in range(3):
+                N, K = pool.shape(mat)
+                pool.pack_into(int(st[e]), mat, inputs.make_weight_fp32_torch(N, K, s, e, mat, dev))
+        x = torch.from_numpy(li.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        lg = torch.from_numpy(li.logits).to(dev)
+        layers.append(dict(li=li, pool=pool, st=torch.from_numpy(st).to(dev), x=x, lg=lg, seed=s))
+    torch.cuda.synchronize()
+    layer = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    # distinct experts per layer (routing is deterministic; used for the algorithmic bytes)
+    distinct = []
+    with torch.cuda.stream(stream):
+        for L in layers:
+            layer.forward(L["x"], L["lg"], L["st"], L["pool"], stream=stream)
+            stream.synchronize()
+            distinct.append(int(torch.unique(layer.ids).numel()))
+
+    def step(i):
+        L = layers[i % R]
+        layer.forward(L["x"], L["lg"], L["st"], L["pool"], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            step(i)
+    stream.synchronize()
+
+    # -------- timed region: device-resident inputs --------
+    _lib.profile_read(reset=True)
+    _lib.profile_enable(True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    _lib.profile_enable(False)
+    prof = _lib.profile_read(reset=True)
+    elapsed_ms = ev0.elapsed_time(ev1)
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+
+    # -------- end to end: pinned host inputs, copies inside the timed region --------
+    host = []
+    for L in layers:
+        host.append((L["x"].cpu().pin_memory(), L["lg"].cpu().pin_memory()))
+    y_host = torch.empty((T, w.H), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(layers[0]["x"])
+    lgd = torch.empty_like(layers[0]["lg"])
+
+    def e2e_step(i):
+        L = layers[i % R]
+        hx, hl = host[i % R]
+        xd.copy_(hx, non_blocking=True)
+        lgd.copy_(hl, non_blocking=True)
+        y = layer.forward(xd, lgd, L["st"], L["pool"], stream=stream)
+        y_host.copy_(y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            e2e_step(i)
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+
+    # -------- roofline of the dominant kernel --------
+    hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    gu = prof["gemm_gate_up"]
+    dn = prof["gemm_down"]
+    dom_name, dom = ("gemm_gate_up", gu) if gu[2] >= dn[2] else ("gemm_down", dn)
+    dom_ms = dom[2] / max(1, dom[1])
+    steps_per_layer = [sum(1 for i in range(args.steps) if i % R == l) for l in range(R)]
+    mean_distinct = sum(d * n for d, n in zip(distinct, steps_per_layer)) / args.steps
+    P = T * w.k
+    flops_step = 6.0 * w.H * w.I * P
+    decode_like = flops_step / (mean_distinct * bytes_per_expert(w.H, w.I)) < 200
+    if dom_name == "gemm_gate_up":
+        alg_bytes = mean_distinct * gate_up_bytes_per_expert(w.H, w.I) + T * w.H * 2 + P * w.I * 2
+        alg_flops = 4.0 * w.H * w.I * P
+    else:
+        alg_bytes = mean_distinct * (w.H * w.I // 2 + w.H * w.I // 16 + 4) + P * w.I * 2 + P * w.H * 2
+        alg_flops = 2.0 * w.H * w.I * P
+    src = os.path.join(ROOT, "moe_expert_layer_renorm_b200", "csrc", "ffn.cu")
+    traffic = traffic_record(src, f"{dom_name}:{args.workload}")
+    if decode_like:
+        achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": traffic, "kernel": dom_name,
+                "launch_ms": round(dom_ms, 5), "algorithmic_bytes": int(alg_bytes), "peak_source": peak_src}
+    else:
+        achieved = alg_flops / (dom_ms * 1e-3) / 1e12
+        peak = bf16_sus
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": dom_name,
+                "launch_ms": round(dom_ms, 5), "algorithmic_flops": alg_flops, "peak_source": peak_src}
+
+    launches = sum(v[0] for v in prof.values())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * T * args.steps / (elapsed_ms * 1e-3)
+    e2e_value = world * T * args.steps / (e2e_ms * 1e-3)
+    layer_gbs = mean_distinct * bytes_per_expert(w.H, w.I) / (ms_per_step * 1e-3) / 1e9
+    layer_tflops = flops_step / (ms_per_step * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(layers[0], w, T, args.cpu_sample_tokens)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 weights, bf16 activations, fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) activations, N(0,sigma) logits, N(0,0.02) weights packed to NVFP4)",
+        "config": {"workload": args.workload, "T": T, "E": w.E, "k": w.k, "H": w.H, "I": w.I,
+                   "route": "softmax_renorm" if w.route_mode == 0 else "topk_softmax",
+                   "slots": w.slots, "layers_rotated": R, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "steps rotate over %d layers; each step reads %.0f MB of expert weights > 126 MB L2"
+                         % (R, mean_distinct * bytes_per_expert(w.H, w.I) / 1e6)},
+        "layer": {"distinct_experts": round(mean_distinct, 2), "weight_GBps": round(layer_gbs, 1),
+                  "TFLOPs": round(layer_tflops, 2), "hbm_frac_of_measured": round(layer_gbs / hbm, 4)},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * w.H * 2 + T * w.E * 4, "d2h_bytes_per_step": T * w.H * 2},
+        "gpu_launches": launches,
+        "kernels": {k: {"launches": v[0], "avg_ms": round(v[2] / v[1], 5) if v[1] else None}
+                    for k, v in prof.items() if v[0]},
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+
+
+def cpu_baseline(L, w, T, n_tokens):
+    """The oracle (as it stands) on a bounded sample of the same layer."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import moe_layer as M
+
+    li = L["li"]
+    pool = L["pool"]
+    st = li.slot_table
+    n = min(T, n_tokens)
+    ids, _ = M.route(li.logits[:n], w.k)
+    exps = {}
+    for e in sorted(set(int(v) for v in ids.reshape(-1))):
+        mats = []
+        for mat in range(3):
+            c, sc, g = pool.tensor_bytes(int(st[e]), mat)
+            N, K = pool.shape(mat)
+            mats.append(M.Nvfp4Tensor(c, sc, g, N, K))
+        exps[e] = M.Expert(*mats)
+    t0 = time.perf_counter()
+    M.moe_layer(li.x_bits[:n], li.logits[:n], w.k, exps, keep_out_perm=False)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} tokens of one {w.name} layer (route, permute, NVFP4 decode of the "
+                      f"{len(exps)} experts they select, fp64 SwiGLU FFN, combine); {dt:.2f} s",
+            "host_cpus": os.cpu_count()}
+
+
+# ------------------------------------------------------ reference arm ---
+
+def run_reference(args):
+    """The CPU oracle timed on the host cores, on this workload's metric."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_info
+
+    from oracle import moe_layer as M
+    from oracle import nvfp4
+
+    w = inputs.WORKLOADS[args.workload]
+    li = inputs.make_layer_inputs(w, 0)
+    s = inputs.layer_seed(w.seed, 0)
+    n = min(w.T, args.cpu_sample_tokens)
+    cache = {}
+
+    def expert(e):
+        if e not in cache:
+            mats = []
+            for mat, (N, K) in enumerate(((w.I, w.H), (w.I, w.H), (w.H, w.I))):
+                c, sc, g = nvfp4.pack(inputs.make_weight_fp32_host(N, K, s, e, mat))
+                mats.append(M.Nvfp4Tensor(c, sc, g, N, K))
+            cache[e] = M.Expert(*mats)
+        return cache[e]
+
+    def step(i):
+        tok = (np.arange(n) + i * n) % w.T
+        ids, _ = M.route(li.logits[tok], w.k)
+        exps = {int(e): expert(int(e)) for e in np.unique(ids)}
+        t0 = time.perf_counter()
+        M.moe_layer(li.x_bits[tok], li.logits[tok], w.k, exps, keep_out_perm=False)
+        return time.perf_counter() - t0
+
+    for i in range(args.warmup):
+        step(i)
+    times = [step(args.warmup + i) for i in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "T": w.T, "E": w.E, "k": w.k, "H": w.H, "I": w.I},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n} tokens of one {w.name} layer per step"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

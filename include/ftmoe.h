@@ -1,0 +1,276 @@
+/*
+ * ftmoe.h -- C ABI of libftmoe.so: one Mixture-of-Experts FFN layer over
+ * NVFP4-quantised experts, for NVIDIA B200 (sm_100a).
+ *
+ * The layer is the hot path of the MoE serving engine described on the
+ * FreeToken pages ("FlashML-org / FreeToken" About page, "Fast Edge-Native
+ * Runtime": MoE serving with a global LRU expert cache and graph-compatible
+ * execution; "FreeToken model guide", MoE expert scheduling strategies and
+ * --quant-backend moe.nvfp4; "sm89-moe-offload" fork README, "Production
+ * configuration" with --moe-cache-size and the wide-load NVFP4 prefill MoE
+ * kernel).  The pages name the pieces but never write the layer down; the
+ * operations below are the plainest reading of a top-k MoE FFN layer:
+ *
+ *   route    -> ft_moe_route      top-k over fp32 router logits, renormalised weights
+ *   permute  -> ft_moe_permute    pairs grouped per expert, expert offsets
+ *   experts  -> ft_moe_ffn_nvfp4  h = silu(Wg x) * (Wu x), o = Wd h, per group
+ *   combine  -> ft_moe_combine    y[t] = sum_j w[t,j] * o[row(t,j)]
+ *   format   -> ft_nvfp4_pack     fp32 weights -> NVFP4 (E2M1 + E4M3/16 + fp32)
+ *   cache    -> ft_slot_*         host LRU of expert slots in a device pool
+ *
+ * Conventions (all functions):
+ *   - Return an int status (FT_OK or a negative FT_ERR_*).  On FT_ERR_CUDA the
+ *     message of the failing runtime call is in ft_last_error() (per thread).
+ *   - Device pointers are plain device addresses; the caller owns every
+ *     buffer (device memory, pinned host memory, workspaces).  No function
+ *     allocates device memory on the hot path.
+ *   - Device work is enqueued on the caller's stream and returns without
+ *     synchronising, except ft_slot_acquire (host LRU bookkeeping) and
+ *     ft_device_status (reads a device word).  Enqueued work never reads the
+ *     host and never synchronises, so a sequence of calls can be captured in
+ *     a CUDA graph.
+ *   - T = 0 is a valid no-op.
+ *   - Kernels never trap: a bad index or an over-long internal wait records
+ *     a code in a per-device status word (FT_DEV_*) and the kernel returns;
+ *     read and clear it with ft_device_status.
+ */
+#ifndef FTMOE_H_
+#define FTMOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FT_API __attribute__((visibility("default")))
+#else
+#define FT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ft_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+enum {
+  FT_OK = 0,
+  FT_ERR_INVALID_ARG = -1,  /* null pointer, k > E, k > 32, E > 1024, bad size or leading dim */
+  FT_ERR_UNSUPPORTED = -2,  /* a shape outside what the kernels support */
+  FT_ERR_CUDA = -3,         /* a CUDA runtime error; see ft_last_error() */
+  FT_ERR_CAPACITY = -4,     /* the slot pool cannot hold the experts one call needs */
+  FT_ERR_NOT_RESIDENT = -5, /* an expert has no host bank registered */
+  FT_ERR_DEVICE = -6,       /* the device status word was set by a kernel */
+};
+
+/* Device status codes recorded by kernels (read with ft_device_status). */
+enum {
+  FT_DEV_OK = 0,
+  FT_DEV_WAIT_TIMEOUT = 1,  /* an internal pipeline wait exceeded ~1 s */
+  FT_DEV_NOT_RESIDENT = 2,  /* a non-empty expert group had slot -1 */
+  FT_DEV_BAD_INDEX = 3,     /* an expert id or slot outside its range */
+};
+
+enum {
+  FT_ROUTE_SOFTMAX_RENORM = 0, /* softmax over all E logits, keep top-k, renormalise */
+  FT_ROUTE_TOPK_SOFTMAX = 1,   /* keep top-k logits, softmax over those k */
+};
+
+enum { FT_GATE = 0, FT_UP = 1, FT_DOWN = 2 };
+
+/*
+ * Where one expert's three NVFP4 tensors live inside a slot of the device
+ * pool (pool + slot * slot_bytes + offset).  Gate and up are [I, H], down is
+ * [H, I] (row = output feature, K contiguous).  For a tensor [N, K]:
+ *   codes   uint8 [N, K/2]       two E2M1 codes per byte, even k in the low nibble
+ *   scales  uint8 [N, ld_scale]  one E4M3 (FN) byte per 16 consecutive k
+ *   global  fp32                 per-tensor scale
+ * value(n,k) = e2m1(code) * e4m3(scale[n][k/16]) * global.
+ * ld_scale is K/16 rounded up to a multiple of 16; all offsets and
+ * slot_bytes are multiples of 256.
+ */
+typedef struct {
+  int32_t H, I;
+  int32_t ld_scale[3];    /* bytes per scale row of gate, up, down */
+  int64_t codes_off[3];
+  int64_t scales_off[3];
+  int64_t global_off[3];
+  int64_t slot_bytes;
+  int32_t num_slots;      /* slots in the pool the layout describes */
+  int32_t reserved;
+} ft_nvfp4_slot_layout;
+
+/* Fill *out with the canonical layout for hidden size H, intermediate I and
+ * num_slots slots.  H and I must be multiples of 64.  Returns FT_OK or
+ * FT_ERR_INVALID_ARG. */
+FT_API int ft_nvfp4_slot_layout_init(int H, int I, int num_slots, ft_nvfp4_slot_layout* out);
+
+/*
+ * Router: per token t, the k experts with the largest logits (descending;
+ * equal logits -> lower expert id first) and their renormalised weights
+ *   w_j = exp(l_j - m) / sum_{i in S} exp(l_i - m),  m = max over S.
+ * mode selects how the fp32 arithmetic is ordered (FT_ROUTE_*); the selected
+ * ids never depend on it.
+ *   logits    device fp32 [T, E] row-major
+ *   topk_ids  device int32 [T, k]  (out)
+ *   topk_w    device fp32  [T, k]  (out)
+ * Requires 1 <= k <= min(E, 32), E <= 1024.
+ */
+FT_API int ft_moe_route(const float* logits, int T, int E, int k, int mode,
+                 int32_t* topk_ids, float* topk_w, ft_stream_t stream);
+
+/*
+ * Permute: pair p = t*k + j (routed to expert topk_ids[p]) is given row
+ * r = expert_offsets[e] + (rank of p among the pairs of e, ascending p).
+ *   expert_offsets  device int32 [E+1]  exclusive prefix sum of group sizes (out)
+ *   perm_src        device int32 [T*k]  row -> pair (out)
+ *   pair_to_row     device int32 [T*k]  pair -> row (out)
+ *   ws              device workspace of ft_moe_permute_workspace_size bytes
+ * Deterministic (no atomics decide any order).  Ids outside [0, E) set
+ * FT_DEV_BAD_INDEX.
+ */
+FT_API int ft_moe_permute(const int32_t* topk_ids, int T, int k, int E,
+                   int32_t* expert_offsets, int32_t* perm_src, int32_t* pair_to_row,
+                   void* ws, size_t ws_bytes, ft_stream_t stream);
+FT_API size_t ft_moe_permute_workspace_size(int T, int k, int E);
+
+/*
+ * Expert FFN over the permuted rows.  For row r of group e (token
+ * t = perm_src[r] / k), with the expert's tensors at
+ * slot_pool + slot_table[e] * layout->slot_bytes:
+ *   h[r]        = silu(gG * (Qg x_t)) * (gU * (Qu x_t))        (I values)
+ *   out_perm[r] = bf16(gD * (Qd h[r]))                          (H values)
+ * where Q* are the E2M1*E4M3 dequantised weights (exact in bf16), g* the
+ * fp32 global scales, products accumulate in fp32 on the tensor cores, and
+ * h is rounded to bf16 before the down projection.
+ *   x              device bf16 [T, H]
+ *   perm_src       device int32 [T*k]     from ft_moe_permute
+ *   expert_offsets device int32 [E+1]     from ft_moe_permute
+ *   slot_table     device int32 [E]       expert -> slot; -1 = not resident
+ *   slot_pool      device, layout->num_slots * layout->slot_bytes bytes, 256-B aligned
+ *   out_perm       device bf16 [T*k, H]   (out)
+ *   ws             device workspace of ft_moe_ffn_workspace_size bytes, 256-B aligned
+ * A non-empty group whose slot is -1 sets FT_DEV_NOT_RESIDENT and its rows are
+ * left unwritten.  H and I must be multiples of 64 and match the layout.
+ */
+FT_API int ft_moe_ffn_nvfp4(const void* x, int T, int H, int I, int E, int k,
+                     const int32_t* perm_src, const int32_t* expert_offsets,
+                     const int32_t* slot_table, const void* slot_pool,
+                     const ft_nvfp4_slot_layout* layout,
+                     void* out_perm, void* ws, size_t ws_bytes, ft_stream_t stream);
+FT_API size_t ft_moe_ffn_workspace_size(int T, int H, int I, int E, int k);
+
+/*
+ * Combine: y[t, :] = bf16( sum_{j<k} topk_w[t,j] * out_perm[pair_to_row[t*k+j], :] ),
+ * summed in fp32 in the order j = 0..k-1.
+ *   out_perm device bf16 [T*k, H], pair_to_row device int32 [T*k],
+ *   topk_w device fp32 [T, k], y device bf16 [T, H] (out).  H % 8 == 0.
+ */
+FT_API int ft_moe_combine(const void* out_perm, const int32_t* pair_to_row, const float* topk_w,
+                   int T, int k, int H, void* y, ft_stream_t stream);
+
+/*
+ * NVFP4 pack of one fp32 tensor [N, K] (K % 16 == 0), every step an IEEE fp32
+ * operation rounded to nearest:
+ *   g   = amax / 2688 (1 if amax = 0)                  -> *global_scale
+ *   s_b = E4M3_rne_sat(amax_b / (6 g))                  per 16-block of a row
+ *   q   = E2M1_rne_sat(w / (e4m3(s_b) * g))             0 where e4m3(s_b) = 0
+ * Ties go to the even code; the code's sign bit follows the input's sign.
+ *   w            device fp32 [N, K]
+ *   codes        device uint8 [N, K/2]       (out; row pitch K/2)
+ *   scales       device uint8 [N, ld_scale]  (out; padding bytes zeroed)
+ *   global_scale device fp32 [1]             (out)
+ *   ws           device workspace, >= 4 bytes (holds amax)
+ * The destinations may point inside a slot (see ft_nvfp4_slot_layout).
+ */
+FT_API int ft_nvfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
+                  float* global_scale, void* ws, ft_stream_t stream);
+
+/*
+ * Read (and optionally clear) the per-device status word of the current
+ * device.  Synchronises the device.  *status receives an FT_DEV_* code.
+ */
+FT_API int ft_device_status(int* status, int clear);
+
+/* ---------------------------------------------------------------------------
+ * Expert slot manager: a host-side LRU over (layer, expert) keys, mirroring
+ * the pages' global LRU expert cache (FreeToken model guide, offload strategy,
+ * OffloadMoeCache with per-(layer, expert) recency and a minimum-size guard;
+ * sm89-moe-offload README, --moe-cache-size).  Each registered expert has a
+ * pinned host copy of its slot image (layout->slot_bytes bytes); a miss is
+ * filled by one cudaMemcpyAsync on the caller's copy stream, and the compute
+ * stream waits on an event recorded after the copies.
+ * ------------------------------------------------------------------------- */
+typedef struct ft_slot_mgr ft_slot_mgr;
+
+typedef struct {
+  int64_t hits, misses, evictions, bytes_h2d;
+} ft_slot_stats_t;
+
+enum {
+  FT_SLOT_DEVICE = 0,    /* normal mode: fills and table uploads on the copy stream */
+  FT_SLOT_HOST_ONLY = 1, /* bookkeeping only: no CUDA calls, device_slot_table is host
+                            memory; for planning and for testing the policy on a host */
+};
+
+/* Manage slots [0, capacity) of device_pool (capacity <= layout->num_slots).
+ * device_pool may be NULL with FT_SLOT_HOST_ONLY. */
+FT_API int ft_slot_create(ft_slot_mgr** mgr, int capacity, const ft_nvfp4_slot_layout* layout,
+                   void* device_pool, int flags);
+/* pinned_src: page-locked host memory of slot_bytes bytes, owned by the caller
+ * and kept alive while the manager exists. */
+FT_API int ft_slot_register_host(ft_slot_mgr* mgr, int layer, int expert, const void* pinned_src);
+/*
+ * Make the n experts host_expert_ids[0..n) of `layer` resident and write
+ * device_slot_table[e] (an int32 [E] device array, E = table_len) for them;
+ * other entries are set to -1.  Resident experts of this call are pinned
+ * until the next acquire; misses evict the least recently used unpinned
+ * slots.  Returns FT_ERR_CAPACITY when more distinct experts are requested
+ * than the pool can hold, FT_ERR_NOT_RESIDENT when a miss has no host bank.
+ * Synchronous on the host; the table upload and fills are enqueued on `copy`
+ * and `compute` waits for them.
+ */
+FT_API int ft_slot_acquire(ft_slot_mgr* mgr, int layer, const int32_t* host_expert_ids, int n,
+                    int32_t* device_slot_table, int table_len, ft_stream_t compute, ft_stream_t copy);
+FT_API int ft_slot_stats(const ft_slot_mgr* mgr, ft_slot_stats_t* out);
+FT_API int ft_slot_destroy(ft_slot_mgr* mgr);
+/* Test hook: make the next `count` host->device fills fail (FT_ERR_CUDA). */
+FT_API int ft_slot_inject_copy_failures(ft_slot_mgr* mgr, int count);
+
+/* ---------------------------------------------------------------------------
+ * Launch accounting and kernel timing.  Every kernel the library launches is
+ * counted by kind.  With timing enabled, CUDA events are recorded around each
+ * launch on its stream (not while the stream is being captured into a graph).
+ * ------------------------------------------------------------------------- */
+enum {
+  FT_KERNEL_ROUTE = 0,
+  FT_KERNEL_PERMUTE = 1,
+  FT_KERNEL_SCHEDULE = 2,
+  FT_KERNEL_GEMM_GATE_UP = 3, /* grouped gate/up GEMM + SwiGLU */
+  FT_KERNEL_GEMM_DOWN = 4,    /* grouped down GEMM */
+  FT_KERNEL_COMBINE = 5,
+  FT_KERNEL_PACK = 6,
+  FT_KERNEL_KINDS = 7,
+};
+
+typedef struct {
+  int64_t launches[FT_KERNEL_KINDS];   /* launches since the last reset */
+  int64_t timed[FT_KERNEL_KINDS];      /* launches that were timed */
+  double total_ms[FT_KERNEL_KINDS];    /* summed device time of the timed launches */
+} ft_profile_t;
+
+/* Turn event timing on (1) or off (0). */
+FT_API int ft_profile_enable(int on);
+/* Synchronise the recorded events, fill *out, and optionally reset. */
+FT_API int ft_profile_read(ft_profile_t* out, int reset);
+
+/* Message of the last FT_ERR_* returned on this thread ("" if none). */
+FT_API const char* ft_last_error(void);
+
+/* Library version string. */
+FT_API const char* ft_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FTMOE_H_ */

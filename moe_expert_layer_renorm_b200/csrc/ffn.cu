@@ -1,0 +1,703 @@
+// Expert FFN over permuted rows: a grouped GEMM with NVFP4 weights on tcgen05.
+//
+// Orientation ("swap AB"): the MMA's M side (128 rows) is 128 output features
+// of one expert's weight matrix and its N side is up to BN permuted token
+// rows of that expert's group, so any group size from 1 row up maps onto one
+// instruction shape (N = group rows rounded up to 16).
+//
+// Data path of one CTA (persistent; 16 warps):
+//   warp 0      TMA: packed E2M1 codes (128 rows x 128 B, 128-byte swizzle)
+//               and E4M3 scales (128 rows x 16 B) of each matrix, 256 K per stage
+//   warps 2-3   cp.async: the unit's token rows (bf16, 64 K per chunk) into
+//               128-byte-swizzled K-major shared memory (the MMA's B operand);
+//               GEMM1 gathers x rows through perm_src, GEMM2 reads h rows
+//   warps 4-11  dequantise one 64-K chunk per step: E2M1 -> f16 (cvt) times the
+//               E4M3 block scale (exact in f16), widened to bf16 (exact), and
+//               stored with tcgen05.st straight into tensor memory, where the
+//               MMA reads it as its A operand (no shared-memory round trip)
+//   warp 1      one thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
+//               accumulators in tensor memory) and commits to the barriers
+//   warps 12-15 epilogue: tcgen05.ld of the accumulators, fp32 global scale,
+//               SwiGLU (GEMM1) and bf16 stores; for split-K, fp32 partials and
+//               a last-arriving-CTA reduction in a fixed order (deterministic)
+//
+// Every pipeline wait is bounded (see sm100.cuh); a wait that gives up sets
+// the device status word and an abort flag, all roles leave their loops, and
+// the CTA drains its outstanding copies and MMAs before freeing tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include "sm100.cuh"
+
+namespace ftmoe {
+
+constexpr int kKW = 256;            // K per weight stage (128 bytes of codes per row)
+constexpr int kKC = 64;             // K per chunk (one 128-byte swizzle atom of bf16)
+constexpr int kCPW = kKW / kKC;     // chunks per weight stage
+constexpr int kCodesBytes = 128 * 128;
+constexpr int kScaleBytes = 128 * 16;
+constexpr int kMatStageBytes = kCodesBytes + kScaleBytes;   // 18 KB, multiple of 1024
+constexpr int kThreads = 512;
+
+struct FfnParams {
+  const __nv_bfloat16* act;   // GEMM1: x [T, K]; GEMM2: h [P, K]
+  const int32_t* perm_src;    // GEMM1: row -> pair (token = pair / k_top); GEMM2: null
+  int k_top;
+  int K;                      // reduction length
+  int M;                      // output features (rows of the weight matrices)
+  int nkw;                    // ceil(K / kKW)
+  int nkc;                    // K / kKC
+  int splits;                 // split-K factor
+  int stages_per_split;
+  const int4* units;          // {expert, m_tile, row_begin, n_rows | split << 16}
+  const int* num_units;
+  const int32_t* slot_table;
+  const uint8_t* pool;
+  long long slot_bytes;
+  long long global_off[2];
+  __nv_bfloat16* out;         // GEMM1: h [P, M]; GEMM2: out_perm [P, M]
+  float* partials;            // split-K partial accumulators
+  int* counters;              // split-K arrival counters, 4 per (tile, m_tile): one per epilogue warp
+};
+
+template <int NMAT, int BN, int WS, int BS, int AS, int DB>
+struct FfnCfg {
+  static constexpr int kWBytes = WS * NMAT * kMatStageBytes;
+  static constexpr int kBStageBytes = BN * 128;
+  static constexpr int kBBytes = BS * kBStageBytes;
+  static constexpr int kNumBars = 2 * WS + 2 * BS + 2 * AS + 2 * DB + 1;
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kWBytes + kBBytes + BN * 4 + kNumBars * 8 + 64;
+  static constexpr int kDCols = DB * NMAT * BN;
+  static constexpr int kTmemCols = kDCols + AS * NMAT * 32;
+  static_assert(kTmemCols <= 512, "tensor memory budget");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+// ------------------------------------------------------------ dequant ---
+
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t v, uint32_t (&q)[4]) {
+  asm("{.reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3]) : "r"(v));
+}
+__device__ __forceinline__ uint32_t e4m3_pair_to_f16x2(uint32_t byte) {   // (s, s)
+  uint32_t r;
+  const uint16_t in = uint16_t(byte | (byte << 8));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(in));
+  return r;
+}
+__device__ __forceinline__ uint32_t hmul2_f16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// f16x2 -> bf16x2 of the same values (exact for E2M1 x E4M3 products: at most
+// 6 significant bits, magnitudes in [2^-10, 2688]).
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
+  uint32_t r;
+  asm("{.reg .b16 a, b;\n .reg .f32 fa, fb;\n mov.b32 {a, b}, %1;\n cvt.f32.f16 fa, a;\n"
+      " cvt.f32.f16 fb, b;\n cvt.rn.bf16x2.f32 %0, fb, fa;\n}"
+      : "=r"(r) : "r"(h));
+  return r;
+}
+
+// 64 codes (two 16-byte words of one row) and their 4 scale bytes -> 32
+// bf16x2 words, word c holding k = 2c (low half) and 2c + 1 (high half).
+__device__ __forceinline__ void dequant_chunk(const uint4& c0, const uint4& c1, uint32_t sc,
+                                              uint32_t (&o)[32]) {
+  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t s2 = e4m3_pair_to_f16x2((sc >> (8 * b)) & 0xFFu);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t q[4];
+      e2m1x8_to_f16x2(w[2 * b + h], q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[(2 * b + h) * 4 + j] = f16x2_to_bf16x2(hmul2_f16(q[j], s2));
+    }
+  }
+}
+
+// ---------------------------------------------------------- pipeline ---
+
+struct Abort {
+  volatile int* flag;
+  __device__ bool wait(uint64_t* bar, uint32_t parity) const {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t n = 0;
+    while (true) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if ((++n & 63u) == 0) {
+        if (*flag) return false;
+        if (globaltimer_ns() - t0 > 1000000000ull) {
+          set_device_status(FT_DEV_WAIT_TIMEOUT);
+          *flag = 1;
+          return false;
+        }
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+template <int NMAT, int BN, int WS, int BS, int AS, int DB>
+__global__ void __launch_bounds__(kThreads, 1)
+ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0,
+                const __grid_constant__ CUtensorMap tm_scales0, const __grid_constant__ CUtensorMap tm_codes1,
+                const __grid_constant__ CUtensorMap tm_scales1) {
+  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* w_smem = smem;
+  uint8_t* b_smem = smem + Cfg::kWBytes;
+  int* rowidx = reinterpret_cast<int*>(b_smem + Cfg::kBBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rowidx + BN);
+  uint64_t* w_full = bars;
+  uint64_t* w_empty = w_full + WS;
+  uint64_t* b_full = w_empty + WS;
+  uint64_t* b_empty = b_full + BS;
+  uint64_t* a_full = b_empty + BS;
+  uint64_t* a_empty = a_full + AS;
+  uint64_t* d_full = a_empty + AS;
+  uint64_t* d_empty = d_full + DB;
+  uint64_t* drain_bar = d_empty + DB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < WS; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], 8); }
+    for (int i = 0; i < BS; ++i) { mbar_init(&b_full[i], 64); mbar_init(&b_empty[i], 1); }
+    for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < DB; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4); }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_codes0); prefetch_tmap(&tm_scales0);
+    if (NMAT > 1) { prefetch_tmap(&tm_codes1); prefetch_tmap(&tm_scales1); }
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Abort ab{abort_flag};
+  const int n_units = *p.num_units;
+  const int nchunks_total = p.nkc;
+
+  auto unit_range = [&](int u, int& e, int& mt, int& rb, int& nr, int& ws0, int& ws1, int& kc0, int& kc1) {
+    const int4 d = p.units[u];
+    e = d.x; mt = d.y; rb = d.z; nr = d.w & 0xFFFF;
+    const int split = d.w >> 16;
+    ws0 = split * p.stages_per_split;
+    ws1 = min(p.nkw, ws0 + p.stages_per_split);
+    kc0 = ws0 * kCPW;
+    kc1 = min(nchunks_total, ws1 * kCPW);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer ---
+    uint32_t wi = 0;
+    if (lane == 0) {
+      const CUtensorMap* tmc[2] = {&tm_codes0, &tm_codes1};
+      const CUtensorMap* tms[2] = {&tm_scales0, &tm_scales1};
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        int e, mt, rb, nr, ws0, ws1, kc0, kc1;
+        unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+        const int slot = __ldg(p.slot_table + e);
+        for (int ws = ws0; ws < ws1; ++ws, ++wi) {
+          const int s = wi % WS;
+          if (!(ok = ab.wait(&w_empty[s], ((wi / WS) & 1) ^ 1))) break;
+          mbar_arrive_expect_tx(&w_full[s], NMAT * kMatStageBytes);
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) {
+            uint8_t* dst = w_smem + (s * NMAT + m) * kMatStageBytes;
+            tma_load_3d(dst, tmc[m], &w_full[s], ws * 128, mt * 128, slot);
+            tma_load_3d(dst + kCodesBytes, tms[m], &w_full[s], ws * 16, mt * 128, slot);
+          }
+        }
+      }
+      // drain: the last copy into every stage buffer has landed
+      for (uint32_t j = (wi > WS ? wi - WS : 0); j < wi; ++j) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&w_full[j % WS], (j / WS) & 1) && globaltimer_ns() - t0 < 1000000000ull) {}
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer ---
+    if (lane == 0) {
+      uint32_t q = 0, di = 0;
+      bool ok = true, issued = false;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++di) {
+        int e, mt, rb, nr, ws0, ws1, kc0, kc1;
+        unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+        const int ds = di % DB;
+        if (!(ok = ab.wait(&d_empty[ds], ((di / DB) & 1) ^ 1))) break;
+        tc_fence_after();
+        const int n_eff = (nr + 15) & ~15;
+        const uint32_t idesc = make_idesc_f16(128, n_eff);
+        for (int c = kc0; c < kc1; ++c, ++q) {
+          const int as = q % AS, bs = q % BS;
+          if (!(ok = ab.wait(&a_full[as], (q / AS) & 1))) break;
+          if (!(ok = ab.wait(&b_full[bs], (q / BS) & 1))) break;
+          tc_fence_after();
+          const uint32_t b_addr = smem_u32(b_smem + bs * Cfg::kBStageBytes);
+#pragma unroll
+          for (int j = 0; j < kKC / 16; ++j) {
+            const uint64_t bdesc = make_sdesc_sw128(b_addr + 32 * j);
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+              const uint32_t d_addr = tmem + (ds * NMAT + m) * BN;
+              const uint32_t a_addr = tmem + Cfg::kDCols + (as * NMAT + m) * 32 + 8 * j;
+              mma_ts_f16(d_addr, a_addr, bdesc, idesc, (c > kc0 || j > 0) ? 1u : 0u);
+            }
+          }
+          issued = true;
+          mma_commit(&a_empty[as]);
+          mma_commit(&b_empty[bs]);
+        }
+        if (!ok) break;
+        mma_commit(&d_full[ds]);
+      }
+      if (issued) {   // drain: every MMA this thread issued has completed
+        mma_commit(drain_bar);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
+      }
+    }
+  } else if (warp < 4) {
+    // --------------------------------------------- B (token) loader ---
+    // Thread tb copies 16-byte column c16 = tb % 8 of rows n = tb / 8 + 8 i.
+    // Up to BS - 1 chunks stay in flight; a chunk's barrier is signalled once
+    // this thread's copies for it have landed.
+    const int tb = threadIdx.x - 64;  // 0..63
+    const int c16 = tb & 7, n_first = tb >> 3;
+    constexpr int kRowsPerThread = BN / 8;
+    constexpr int kLag = BS - 1;
+    uint32_t q = 0, pending = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      int e, mt, rb, nr, ws0, ws1, kc0, kc1;
+      unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+      int rows[kRowsPerThread];
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int n = n_first + 8 * i;
+        rows[i] = n < nr ? (p.perm_src ? __ldg(p.perm_src + rb + n) / p.k_top : rb + n) : -1;
+      }
+      const int n_eff = (nr + 15) & ~15;
+      for (int c = kc0; c < kc1; ++c, ++q) {
+        const int bs = q % BS;
+        if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&b_empty[bs], ((q / BS) & 1) ^ 1)))) break;
+        const uint32_t dst0 = smem_u32(b_smem + bs * Cfg::kBStageBytes);
+        const int kk = c * kKC + c16 * 8;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int n = n_first + 8 * i;
+          if (n < n_eff) {
+            const bool live = rows[i] >= 0 && kk < p.K;
+            const __nv_bfloat16* src = live ? p.act + size_t(rows[i]) * p.K + kk : p.act;
+            cp_async_16(dst0 + n * 128 + ((c16 ^ (n & 7)) << 4), src, live ? 16u : 0u);
+          }
+        }
+        cp_async_commit();
+        if (++pending > kLag) {
+          cp_async_wait<kLag>();
+          fence_proxy_async_smem();
+          mbar_arrive(&b_full[(q - kLag) % BS]);
+          --pending;
+        }
+      }
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    for (; pending > 0; --pending) mbar_arrive(&b_full[(q - pending) % BS]);
+  } else if (warp < 12) {
+    // -------------------------------------------------- dequantise ---
+    const int g = (warp - 4) >> 2;            // warpgroup: even / odd chunks
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;      // weight row within the tile = TMEM lane
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    uint32_t q = 0, wi = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      int e, mt, rb, nr, ws0, ws1, kc0, kc1;
+      unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+      for (int ws = ws0; ws < ws1 && ok; ++ws, ++wi) {
+        const int s = wi % WS;
+        if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&w_full[s], (wi / WS) & 1)))) break;
+        const int c_end = min(kc1, (ws + 1) * kCPW);
+        for (int c = ws * kCPW; c < c_end; ++c, ++q) {
+          if ((q & 1) != uint32_t(g)) continue;
+          const int as = q % AS;
+          if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&a_empty[as], ((q / AS) & 1) ^ 1)))) break;
+          tc_fence_after();
+          const int cc = c - ws * kCPW;
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) {
+            const uint8_t* base = w_smem + (s * NMAT + m) * kMatStageBytes;
+            const uint8_t* crow = base + row * 128;
+            const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2 * cc) ^ (row & 7)) << 4));
+            const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2 * cc + 1) ^ (row & 7)) << 4));
+            const uint32_t sc = *reinterpret_cast<const uint32_t*>(base + kCodesBytes + row * 16 + cc * 4);
+            uint32_t o[32];
+            dequant_chunk(c0, c1, sc, o);
+            tmem_st_32x32b_x32(tmem + lane_base + Cfg::kDCols + (as * NMAT + m) * 32, o);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[as]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&w_empty[s]);
+      }
+    }
+  } else {
+    // ---------------------------------------------------- epilogue ---
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    uint32_t di = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++di) {
+      int e, mt, rb, nr, ws0, ws1, kc0, kc1;
+      unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+      const int ds = di % DB;
+      const int feat = mt * 128 + row;
+      const int slot = __ldg(p.slot_table + e);
+      const uint8_t* sbase = p.pool + size_t(slot) * size_t(p.slot_bytes);
+      float gsc[NMAT];
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) gsc[m] = __ldg(reinterpret_cast<const float*>(sbase + p.global_off[m]));
+      if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&d_full[ds], (di / DB) & 1)))) break;
+      tc_fence_after();
+      const int n_eff = (nr + 15) & ~15;
+      const bool split = p.splits > 1;
+      for (int n0 = 0; n0 < n_eff; n0 += 16) {
+        uint32_t v[NMAT][16];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) tmem_ld_32x32b_x16(tmem + lane_base + (ds * NMAT + m) * BN + n0, v[m]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int n = n0 + i;
+          if (n >= nr) break;
+          if (split) {
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+              p.partials[(size_t(u) * NMAT + m) * 128 * BN + size_t(n) * 128 + row] = __uint_as_float(v[m][i]);
+          } else if (feat < p.M) {
+            float r;
+            if (NMAT == 2) r = silu_mul(gsc[0] * __uint_as_float(v[0][i]), gsc[NMAT - 1] * __uint_as_float(v[NMAT - 1][i]));
+            else r = gsc[0] * __uint_as_float(v[0][i]);
+            p.out[size_t(rb + n) * p.M + feat] = __float2bfloat16_rn(r);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[ds]);
+      if (split) {
+        // this warp's 32 rows: the last of the `splits` warps to arrive sums
+        // the partials in split order and writes the result
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = atomicAdd(p.counters + (u / p.splits) * 4 + quarter, 1) == p.splits - 1;
+        last = __shfl_sync(0xFFFFFFFFu, last, 0);
+        if (last) {
+          __threadfence();
+          const int u0 = u - (p.units[u].w >> 16);
+          for (int n = 0; n < nr; ++n) {
+            float acc[NMAT];
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) acc[m] = 0.0f;
+            for (int sp = 0; sp < p.splits; ++sp) {
+#pragma unroll
+              for (int m = 0; m < NMAT; ++m)
+                acc[m] += __ldcg(p.partials + (size_t(u0 + sp) * NMAT + m) * 128 * BN + size_t(n) * 128 + row);
+            }
+            if (feat < p.M) {
+              float r;
+              if (NMAT == 2) r = silu_mul(gsc[0] * acc[0], gsc[NMAT - 1] * acc[NMAT - 1]);
+              else r = gsc[0] * acc[0];
+              p.out[size_t(rb + n) * p.M + feat] = __float2bfloat16_rn(r);
+            }
+          }
+          if (lane == 0) p.counters[(u / p.splits) * 4 + quarter] = 0;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------- schedule ---
+
+__device__ int block_exclusive_scan(int v, int* smem_warp_sums);
+
+// Builds both GEMMs' work lists from the expert offsets (one CTA; E <= 1024).
+// Unit u = ((tile * m_tiles) + m_tile) * splits + split, tiles numbered in
+// expert order, so the splits of one output tile are consecutive.
+__global__ void __launch_bounds__(1024) ffn_schedule_kernel(
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ slot_table, int E, int num_slots,
+    int bn1, int mt1, int s1, int bn2, int mt2, int s2, int4* __restrict__ units1, int4* __restrict__ units2,
+    int* __restrict__ counts, int* __restrict__ counters1, int ncnt1, int* __restrict__ counters2, int ncnt2) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  int n = 0, rb = 0;
+  if (e < E) {
+    rb = offsets[e];
+    n = offsets[e + 1] - rb;
+    if (n > 0) {
+      const int slot = slot_table[e];
+      if (slot < 0) { set_device_status(FT_DEV_NOT_RESIDENT); n = 0; }
+      else if (slot >= num_slots) { set_device_status(FT_DEV_BAD_INDEX); n = 0; }
+    }
+  }
+  const int t1 = (n + bn1 - 1) / bn1, t2 = (n + bn2 - 1) / bn2;
+  const int ex1 = block_exclusive_scan(t1, warp_sums);
+  const int ex2 = block_exclusive_scan(t2, warp_sums);
+  for (int t = 0; t < t1; ++t)
+    for (int m = 0; m < mt1; ++m)
+      for (int s = 0; s < s1; ++s)
+        units1[((ex1 + t) * mt1 + m) * s1 + s] = make_int4(e, m, rb + t * bn1, min(bn1, n - t * bn1) | (s << 16));
+  for (int t = 0; t < t2; ++t)
+    for (int m = 0; m < mt2; ++m)
+      for (int s = 0; s < s2; ++s)
+        units2[((ex2 + t) * mt2 + m) * s2 + s] = make_int4(e, m, rb + t * bn2, min(bn2, n - t * bn2) | (s << 16));
+  if (e == blockDim.x - 1) {
+    counts[0] = (ex1 + t1) * mt1 * s1;
+    counts[1] = (ex2 + t2) * mt2 * s2;
+  }
+  for (int i = threadIdx.x; i < ncnt1; i += blockDim.x) counters1[i] = 0;
+  for (int i = threadIdx.x; i < ncnt2; i += blockDim.x) counters2[i] = 0;
+}
+
+// --------------------------------------------------------------- host ---
+
+struct GemmShape { int bn, splits, sps, ws, bs, as, db; };
+
+struct FfnPlan {
+  bool decode;
+  GemmShape g1, g2;
+  int mt1, mt2, nkw1, nkw2, nkc1, nkc2;
+  long long max_tiles1, max_tiles2;
+  // workspace layout (byte offsets)
+  size_t off_h, off_units1, off_units2, off_counts, off_cnt1, off_cnt2, off_part1, off_part2, total;
+  long long max_units1, max_units2;
+};
+
+static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int choose_splits(double units_est, int nkw, int num_sms, int* sps_out) {
+  int s = 1;
+  if (units_est < num_sms) s = (int)ceil(num_sms / units_est);
+  s = std::max(1, std::min(s, nkw));
+  const int sps = (nkw + s - 1) / s;
+  *sps_out = sps;
+  return (nkw + sps - 1) / sps;
+}
+
+static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
+  FfnPlan pl{};
+  const long long P = (long long)T * k;
+  const double distinct = E * (1.0 - pow(1.0 - double(k) / E, double(T)));
+  const double mean_rows = distinct > 0 ? double(P) / distinct : 0.0;
+  pl.decode = mean_rows <= 32.0;
+  pl.mt1 = (I + 127) / 128;
+  pl.mt2 = (H + 127) / 128;
+  pl.nkw1 = (H + kKW - 1) / kKW;
+  pl.nkw2 = (I + kKW - 1) / kKW;
+  pl.nkc1 = H / kKC;
+  pl.nkc2 = I / kKC;
+  if (pl.decode) {
+    pl.g1 = {32, 1, 0, 5, 4, 4, 2};
+    pl.g2 = {32, 1, 0, 8, 4, 4, 2};
+  } else {
+    pl.g1 = {128, 1, 0, 3, 4, 4, 1};
+    pl.g2 = {128, 1, 0, 3, 6, 4, 2};
+  }
+  const double est_tiles1 = std::max(1.0, ceil(distinct) + (pl.decode ? 0.0 : double(P) / pl.g1.bn));
+  const double est_tiles2 = std::max(1.0, ceil(distinct) + (pl.decode ? 0.0 : double(P) / pl.g2.bn));
+  pl.g1.splits = choose_splits(est_tiles1 * pl.mt1, pl.nkw1, num_sms, &pl.g1.sps);
+  pl.g2.splits = choose_splits(est_tiles2 * pl.mt2, pl.nkw2, num_sms, &pl.g2.sps);
+  const long long active = std::min<long long>(E, P);
+  pl.max_tiles1 = active + P / pl.g1.bn;
+  pl.max_tiles2 = active + P / pl.g2.bn;
+  pl.max_units1 = pl.max_tiles1 * pl.mt1 * pl.g1.splits;
+  pl.max_units2 = pl.max_tiles2 * pl.mt2 * pl.g2.splits;
+  size_t o = 0;
+  pl.off_h = o;       o = align256(o + size_t(P) * I * 2);
+  pl.off_units1 = o;  o = align256(o + size_t(pl.max_units1) * 16);
+  pl.off_units2 = o;  o = align256(o + size_t(pl.max_units2) * 16);
+  pl.off_counts = o;  o = align256(o + 16);
+  pl.off_cnt1 = o;    o = align256(o + size_t(pl.max_tiles1 * pl.mt1) * 4 * 4);
+  pl.off_cnt2 = o;    o = align256(o + size_t(pl.max_tiles2 * pl.mt2) * 4 * 4);
+  pl.off_part1 = o;
+  if (pl.g1.splits > 1) o = align256(o + size_t(pl.max_units1) * 2 * 128 * pl.g1.bn * 4);
+  pl.off_part2 = o;
+  if (pl.g2.splits > 1) o = align256(o + size_t(pl.max_units2) * 1 * 128 * pl.g2.bn * 4);
+  pl.total = o;
+  return pl;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// codes: [rows, K/2] bytes per slot, 128 x 128-byte boxes, 128-byte swizzle.
+// scales: [rows, ld_scale] bytes per slot, 128 x 16-byte boxes.
+static bool make_weight_maps(const uint8_t* pool, const ft_nvfp4_slot_layout& L, int mat, int rows, int K,
+                             CUtensorMap* codes, CUtensorMap* scales) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  {
+    const cuuint64_t dims[3] = {cuuint64_t(K / 2), cuuint64_t(rows), cuuint64_t(L.num_slots)};
+    const cuuint64_t strides[2] = {cuuint64_t(K / 2), cuuint64_t(L.slot_bytes)};
+    const cuuint32_t box[3] = {128, 128, 1};
+    if (enc(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)(pool + L.codes_off[mat]), dims, strides, box,
+            elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  {
+    const cuuint64_t dims[3] = {cuuint64_t(L.ld_scale[mat]), cuuint64_t(rows), cuuint64_t(L.num_slots)};
+    const cuuint64_t strides[2] = {cuuint64_t(L.ld_scale[mat]), cuuint64_t(L.slot_bytes)};
+    const cuuint32_t box[3] = {16, 128, 1};
+    if (enc(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)(pool + L.scales_off[mat]), dims, strides, box,
+            elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
+template <int NMAT, int BN, int WS, int BS, int AS, int DB>
+static cudaError_t launch_gemm(const FfnParams& p, int grid, const CUtensorMap& c0, const CUtensorMap& s0,
+                               const CUtensorMap& c1, const CUtensorMap& s1, cudaStream_t s) {
+  ProfileScope prof(NMAT == 2 ? FT_KERNEL_GEMM_GATE_UP : FT_KERNEL_GEMM_DOWN, s);
+  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB>;
+  auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<grid, kThreads, Cfg::kSmemBytes, s>>>(p, c0, s0, c1, s1);
+  return cudaGetLastError();
+}
+
+static int device_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, const int32_t* perm_src,
+                              const int32_t* offsets, const int32_t* slot_table, const void* pool_v,
+                              const ft_nvfp4_slot_layout& L, void* out_perm, void* ws, cudaStream_t s,
+                              const char** why) {
+  const int num_sms = device_sm_count();
+  const FfnPlan pl = plan_ffn(T, H, I, E, k, num_sms);
+  const uint8_t* pool = static_cast<const uint8_t*>(pool_v);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  CUtensorMap tmc[3], tms[3];
+  const int rows[3] = {I, I, H}, Ks[3] = {H, H, I};
+  for (int m = 0; m < 3; ++m)
+    if (!make_weight_maps(pool, L, m, rows[m], Ks[m], &tmc[m], &tms[m])) {
+      *why = "cuTensorMapEncodeTiled failed for the slot pool";
+      return cudaErrorInvalidValue;
+    }
+  int4* units1 = reinterpret_cast<int4*>(w + pl.off_units1);
+  int4* units2 = reinterpret_cast<int4*>(w + pl.off_units2);
+  int* counts = reinterpret_cast<int*>(w + pl.off_counts);
+  int* cnt1 = reinterpret_cast<int*>(w + pl.off_cnt1);
+  int* cnt2 = reinterpret_cast<int*>(w + pl.off_cnt2);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(w + pl.off_h);
+  {
+  ProfileScope prof(FT_KERNEL_SCHEDULE, s);
+  ffn_schedule_kernel<<<1, 1024, 0, s>>>(offsets, slot_table, E, L.num_slots, pl.g1.bn, pl.mt1, pl.g1.splits,
+                                         pl.g2.bn, pl.mt2, pl.g2.splits, units1, units2, counts, cnt1,
+                                         int(pl.max_tiles1 * pl.mt1 * 4), cnt2, int(pl.max_tiles2 * pl.mt2 * 4));
+  }
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+
+  FfnParams p1{};
+  p1.act = static_cast<const __nv_bfloat16*>(x);
+  p1.perm_src = perm_src;
+  p1.k_top = k;
+  p1.K = H;
+  p1.M = I;
+  p1.nkw = pl.nkw1;
+  p1.nkc = pl.nkc1;
+  p1.splits = pl.g1.splits;
+  p1.stages_per_split = pl.g1.sps;
+  p1.units = units1;
+  p1.num_units = counts;
+  p1.slot_table = slot_table;
+  p1.pool = pool;
+  p1.slot_bytes = L.slot_bytes;
+  p1.global_off[0] = L.global_off[FT_GATE];
+  p1.global_off[1] = L.global_off[FT_UP];
+  p1.out = h;
+  p1.partials = reinterpret_cast<float*>(w + pl.off_part1);
+  p1.counters = cnt1;
+  const int grid1 = int(std::min<long long>(num_sms, pl.max_units1));
+
+  FfnParams p2 = p1;
+  p2.act = h;
+  p2.perm_src = nullptr;
+  p2.K = I;
+  p2.M = H;
+  p2.nkw = pl.nkw2;
+  p2.nkc = pl.nkc2;
+  p2.splits = pl.g2.splits;
+  p2.stages_per_split = pl.g2.sps;
+  p2.units = units2;
+  p2.num_units = counts + 1;
+  p2.global_off[0] = L.global_off[FT_DOWN];
+  p2.global_off[1] = L.global_off[FT_DOWN];
+  p2.out = static_cast<__nv_bfloat16*>(out_perm);
+  p2.partials = reinterpret_cast<float*>(w + pl.off_part2);
+  p2.counters = cnt2;
+  const int grid2 = int(std::min<long long>(num_sms, pl.max_units2));
+
+  if (pl.decode) {
+    err = launch_gemm<2, 32, 5, 4, 4, 2>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], s);
+    if (err == cudaSuccess) err = launch_gemm<1, 32, 8, 4, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], s);
+  } else {
+    err = launch_gemm<2, 128, 3, 4, 4, 1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], s);
+    if (err == cudaSuccess) err = launch_gemm<1, 128, 3, 6, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], s);
+  }
+  return err;
+}
+
+}  // namespace ftmoe

@@ -1,0 +1,109 @@
+// NVFP4 pack of an fp32 tensor [N, K]: per-tensor fp32 scale, one E4M3 scale
+// per 16 consecutive K of a row, two E2M1 codes per byte (even k low nibble).
+// Every step is an IEEE fp32 operation rounded to nearest (no fast math):
+//   g   = amax / 2688 (1 if amax == 0)
+//   s_b = e4m3_rn_satfinite(amax_b / (6 g))
+//   q   = e2m1_rn_satfinite(w / (e4m3(s_b) g)),  0 where e4m3(s_b) == 0
+// The conversions to E4M3/E2M1 use the hardware cvt (round to nearest even,
+// saturate to the largest finite value).
+#include <cuda_fp16.h>
+#include "sm100.cuh"
+
+namespace ftmoe {
+
+__global__ void __launch_bounds__(256) amax_kernel(const float4* __restrict__ w, long long n4,
+                                                   unsigned int* __restrict__ amax_bits) {
+  float m = 0.0f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 v = __ldg(w + i);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));  // m >= 0: bits order like values
+}
+
+__device__ __forceinline__ uint32_t cvt_e4m3_satfinite(float r) {  // r >= 0
+  uint16_t pair;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(0.0f), "f"(r));
+  return pair & 0xFFu;  // second source lands in the low byte
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+  uint32_t h2;
+  const uint16_t in = uint16_t(byte);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return __half2float(__ushort_as_half(uint16_t(h2 & 0xFFFFu)));
+}
+
+// two fp32 -> one byte of two E2M1 codes: `lo` in bits 3..0, `hi` in bits 7..4
+__device__ __forceinline__ uint32_t cvt_e2m1x2_satfinite(float lo, float hi) {
+  uint32_t out;
+  asm("{.reg .b8 b;\n cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n cvt.u32.u8 %0, b;\n}"
+      : "=r"(out) : "f"(hi), "f"(lo));
+  return out & 0xFFu;
+}
+
+// One thread per 16-element block.
+__global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ w, int N, int K,
+                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                   int ld_scale, const unsigned int* __restrict__ amax_bits,
+                                                   float* __restrict__ global_scale) {
+  const int nb = K / 16;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const float amax = __uint_as_float(*amax_bits);
+  const float g = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+  if (i == 0) *global_scale = g;
+  if (i >= (long long)N * ld_scale) return;
+  const int n = int(i / ld_scale), b = int(i % ld_scale);
+  if (b >= nb) {  // scale-row padding
+    scales[size_t(n) * ld_scale + b] = 0;
+    return;
+  }
+  const float4* src = reinterpret_cast<const float4*>(w + size_t(n) * K + size_t(b) * 16);
+  float v[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 f = __ldg(src + q);
+    v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+  }
+  float amax_b = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) amax_b = fmaxf(amax_b, fabsf(v[q]));
+  const float denom = __fmul_rn(6.0f, g);
+  const uint32_t sbyte = cvt_e4m3_satfinite(__fdiv_rn(amax_b, denom));
+  const float sd = e4m3_to_f32(sbyte);
+  const float qden = __fmul_rn(sd, g);
+  uint32_t words[2] = {0u, 0u};
+  if (sd != 0.0f) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t byte = cvt_e2m1x2_satfinite(__fdiv_rn(v[2 * q], qden), __fdiv_rn(v[2 * q + 1], qden));
+      words[q / 4] |= byte << (8 * (q % 4));
+    }
+  }
+  uint2* dst = reinterpret_cast<uint2*>(codes + size_t(n) * (K / 2) + size_t(b) * 8);
+  *dst = make_uint2(words[0], words[1]);
+  scales[size_t(n) * ld_scale + b] = uint8_t(sbyte);
+}
+
+static cudaError_t launch_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
+                               float* global_scale, void* ws, cudaStream_t s) {
+  unsigned int* amax = static_cast<unsigned int*>(ws);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), s);
+  if (e != cudaSuccess) return e;
+  const long long n4 = (long long)N * K / 4;
+  const int blocks1 = int(std::min<long long>((n4 + 255) / 256, 148LL * 8));
+  {
+    ProfileScope prof(FT_KERNEL_PACK, s);
+    amax_kernel<<<blocks1, 256, 0, s>>>(reinterpret_cast<const float4*>(w), n4, amax);
+  }
+  const long long nthreads = (long long)N * ld_scale;
+  ProfileScope prof(FT_KERNEL_PACK, s);
+  pack_kernel<<<dim3(unsigned((nthreads + 255) / 256)), 256, 0, s>>>(w, N, K, codes, scales, ld_scale, amax,
+                                                                       global_scale);
+  return cudaGetLastError();
+}
+
+}  // namespace ftmoe

@@ -1,0 +1,177 @@
+// Permute: a stable counting sort of the T*k (token, rank) pairs by expert.
+//
+// Pairs are cut into chunks of CHUNK consecutive pair indices.
+//   1. per-chunk histograms of the expert ids            (one CTA per chunk)
+//   2. expert offsets = exclusive scan of the totals, and
+//      base[c][e] = offsets[e] + sum_{c' < c} count[c'][e] (one CTA)
+//   3. scatter: one warp walks its chunk 32 pairs at a time; pairs of the same
+//      expert inside a step are ranked with __match_any_sync, so a pair's row
+//      is base + (number of earlier pairs of its expert).  No atomic decides
+//      any order, so the result is deterministic.
+// Small inputs (one chunk) run all three steps in a single CTA.
+#include "sm100.cuh"
+
+namespace ftmoe {
+
+constexpr int kPermChunk = 1024;
+constexpr int kMaxExperts = 1024;
+
+__device__ __forceinline__ bool valid_expert(int e, int E) { return e >= 0 && e < E; }
+
+// Block-wide exclusive scan of one int per thread over blockDim.x <= 1024 threads.
+__device__ int block_exclusive_scan(int v, int* smem_warp_sums) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = (blockDim.x + 31) >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) smem_warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < nwarps ? smem_warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, s, off);
+      if (lane >= off) s += y;
+    }
+    if (lane < nwarps) smem_warp_sums[lane] = s;  // inclusive
+  }
+  __syncthreads();
+  const int before = warp > 0 ? smem_warp_sums[warp - 1] : 0;
+  __syncthreads();
+  return before + x - v;
+}
+
+// Walk pairs [p0, p1) in order with one warp; cursor[e] is this chunk's next
+// row for expert e (shared memory), advanced as pairs are placed.
+__device__ void scatter_chunk_warp(const int32_t* __restrict__ ids, int p0, int p1, int E, int* cursor,
+                                   int32_t* __restrict__ perm_src, int32_t* __restrict__ pair_to_row,
+                                   int P) {
+  const int lane = threadIdx.x & 31;
+  for (int base = p0; base < p1; base += 32) {
+    const int p = base + lane;
+    const bool live = p < p1;
+    int e = live ? __ldg(ids + p) : -1;
+    if (live && !valid_expert(e, E)) { set_device_status(FT_DEV_BAD_INDEX); e = -1; }
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int leader = __ffs(peers) - 1;
+    int row = -1;
+    if (e >= 0) row = cursor[e] + rank;
+    __syncwarp();
+    if (e >= 0 && lane == leader) cursor[e] += __popc(peers);
+    __syncwarp();
+    if (e >= 0 && row >= 0 && row < P) {
+      perm_src[row] = p;
+      pair_to_row[p] = row;
+    }
+  }
+}
+
+// Whole permutation in one CTA (P <= kPermChunk).
+__global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                             int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ perm_src,
+                                                             int32_t* __restrict__ pair_to_row) {
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int warp_sums[32];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < P; p += blockDim.x) {
+    const int e = __ldg(ids + p);
+    if (valid_expert(e, E)) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  // E <= 1024 = blockDim.x: one expert per thread
+  const int e = threadIdx.x;
+  const int c = e < E ? cnt[e] : 0;
+  const int ex = block_exclusive_scan(c, warp_sums);
+  if (e < E) { offsets[e] = ex; cnt[e] = ex; }
+  if (e == E - 1) offsets[E] = ex + c;
+  __syncthreads();
+  if (threadIdx.x < 32) scatter_chunk_warp(ids, 0, P, E, cnt, perm_src, pair_to_row, P);
+}
+
+__global__ void __launch_bounds__(256) permute_hist_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                           int32_t* __restrict__ counts) {
+  __shared__ int cnt[kMaxExperts];
+  const int c = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
+  for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+    const int e = __ldg(ids + p);
+    if (valid_expert(e, E)) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[size_t(c) * E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ counts, int nchunks, int E,
+                                                            int32_t* __restrict__ offsets) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E)
+    for (int c = 0; c < nchunks; ++c) total += counts[size_t(c) * E + e];
+  const int ex = block_exclusive_scan(total, warp_sums);
+  if (e < E) {
+    offsets[e] = ex;
+    int run = ex;
+    for (int c = 0; c < nchunks; ++c) {  // counts become per-chunk base rows
+      const int n = counts[size_t(c) * E + e];
+      counts[size_t(c) * E + e] = run;
+      run += n;
+    }
+  }
+  if (e == E - 1) offsets[E] = ex + total;
+}
+
+__global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                              const int32_t* __restrict__ bases,
+                                                              int32_t* __restrict__ perm_src,
+                                                              int32_t* __restrict__ pair_to_row) {
+  __shared__ int cursor[kMaxExperts];
+  const int c = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] = bases[size_t(c) * E + e];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
+    scatter_chunk_warp(ids, p0, p1, E, cursor, perm_src, pair_to_row, P);
+  }
+}
+
+static size_t permute_ws_bytes(int T, int k, int E) {
+  const long long P = (long long)T * k;
+  const long long nchunks = (P + kPermChunk - 1) / kPermChunk;
+  return nchunks <= 1 ? 0 : size_t(nchunks) * E * sizeof(int32_t);
+}
+
+static cudaError_t launch_permute(const int32_t* ids, int T, int k, int E, int32_t* offsets,
+                                  int32_t* perm_src, int32_t* pair_to_row, void* ws, cudaStream_t s) {
+  const int P = T * k;
+  const int nchunks = (P + kPermChunk - 1) / kPermChunk;
+  if (nchunks <= 1) {
+    ProfileScope prof(FT_KERNEL_PERMUTE, s);
+    permute_small_kernel<<<1, 1024, 0, s>>>(ids, P, E, offsets, perm_src, pair_to_row);
+    return cudaGetLastError();
+  }
+  int32_t* counts = static_cast<int32_t*>(ws);
+  {
+    ProfileScope prof(FT_KERNEL_PERMUTE, s);
+    permute_hist_kernel<<<nchunks, 256, 0, s>>>(ids, P, E, counts);
+  }
+  {
+    ProfileScope prof(FT_KERNEL_PERMUTE, s);
+    permute_scan_kernel<<<1, 1024, 0, s>>>(counts, nchunks, E, offsets);
+  }
+  {
+    ProfileScope prof(FT_KERNEL_PERMUTE, s);
+    permute_scatter_kernel<<<nchunks, 256, 0, s>>>(ids, P, E, counts, perm_src, pair_to_row);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ftmoe

@@ -1,0 +1,250 @@
+// Expert slot manager: a host-side LRU over (layer, expert) keys whose values
+// are slots of a caller-owned device pool.  It mirrors the engine's global
+// LRU expert cache (FreeToken model guide, offload strategy: OffloadMoeCache
+// with per-(layer, expert) recency and a guard that refuses a cache too small
+// to make progress; sm89-moe-offload README, --moe-cache-size).
+//
+// acquire(layer, ids):
+//   1. every requested expert that is resident is a hit: it moves to the
+//      most-recently-used end and is pinned for this call;
+//   2. every miss takes a free slot, else evicts the least recently used
+//      slot not pinned by this call, and is filled from its pinned host bank
+//      with one cudaMemcpyAsync on the copy stream;
+//   3. the device slot table [E] is uploaded on the copy stream, an event is
+//      recorded there and the compute stream waits on it.
+// More distinct experts than capacity -> FT_ERR_CAPACITY (nothing changes).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <list>
+#include <mutex>
+#include <unordered_map>
+#include <vector>
+
+#include "ftmoe.h"
+
+namespace ftmoe {
+void set_last_error(const char* msg);
+}
+
+struct ft_slot_mgr {
+  int capacity = 0;
+  ft_nvfp4_slot_layout layout{};
+  uint8_t* pool = nullptr;
+  // LRU list of resident keys, most recent at the front
+  std::list<uint64_t> lru;
+  struct Entry {
+    int slot;
+    std::list<uint64_t>::iterator it;
+  };
+  std::unordered_map<uint64_t, Entry> resident;
+  std::unordered_map<uint64_t, const void*> banks;
+  std::vector<int> free_slots;
+  std::vector<int32_t> host_table;      // staging copy of the last uploaded table
+  int32_t* pinned_table = nullptr;      // page-locked staging for the async upload
+  int pinned_table_len = 0;
+  cudaEvent_t done = nullptr;
+  cudaEvent_t compute_mark = nullptr;   // compute-stream position when a fill evicts a slot
+  ft_slot_stats_t stats{};
+  int inject_failures = 0;
+  bool host_only = false;               // FT_SLOT_HOST_ONLY: bookkeeping only, no CUDA calls
+  std::mutex mu;
+};
+
+static inline uint64_t slot_key(int layer, int expert) {
+  return (uint64_t(uint32_t(layer)) << 32) | uint32_t(expert);
+}
+
+extern "C" int ft_slot_create(ft_slot_mgr** mgr, int capacity, const ft_nvfp4_slot_layout* layout,
+                              void* device_pool, int flags) {
+  const bool host_only = (flags & FT_SLOT_HOST_ONLY) != 0;
+  if (!mgr || !layout || (!device_pool && !host_only) || capacity <= 0 || capacity > layout->num_slots) {
+    ftmoe::set_last_error("ft_slot_create: bad argument");
+    return FT_ERR_INVALID_ARG;
+  }
+  auto* m = new ft_slot_mgr();
+  m->capacity = capacity;
+  m->layout = *layout;
+  m->pool = static_cast<uint8_t*>(device_pool);
+  m->host_only = host_only;
+  for (int s = capacity - 1; s >= 0; --s) m->free_slots.push_back(s);
+  if (!host_only && (cudaEventCreateWithFlags(&m->done, cudaEventDisableTiming) != cudaSuccess ||
+                     cudaEventCreateWithFlags(&m->compute_mark, cudaEventDisableTiming) != cudaSuccess)) {
+    ftmoe::set_last_error("ft_slot_create: cudaEventCreate failed");
+    delete m;
+    return FT_ERR_CUDA;
+  }
+  *mgr = m;
+  return FT_OK;
+}
+
+extern "C" int ft_slot_register_host(ft_slot_mgr* m, int layer, int expert, const void* pinned_src) {
+  if (!m || !pinned_src || layer < 0 || expert < 0) {
+    ftmoe::set_last_error("ft_slot_register_host: bad argument");
+    return FT_ERR_INVALID_ARG;
+  }
+  std::lock_guard<std::mutex> g(m->mu);
+  m->banks[slot_key(layer, expert)] = pinned_src;
+  return FT_OK;
+}
+
+extern "C" int ft_slot_inject_copy_failures(ft_slot_mgr* m, int count) {
+  if (!m || count < 0) return FT_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> g(m->mu);
+  m->inject_failures = count;
+  return FT_OK;
+}
+
+extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, int n, int32_t* device_table,
+                               int table_len, ft_stream_t compute, ft_stream_t copy) {
+  if (!m || (n > 0 && !ids) || !device_table || table_len <= 0 || n < 0) {
+    ftmoe::set_last_error("ft_slot_acquire: bad argument");
+    return FT_ERR_INVALID_ARG;
+  }
+  std::lock_guard<std::mutex> g(m->mu);
+  // distinct requested experts, in request order
+  std::vector<int> want;
+  want.reserve(n);
+  {
+    std::vector<char> seen(table_len, 0);
+    for (int i = 0; i < n; ++i) {
+      const int e = ids[i];
+      if (e < 0 || e >= table_len) {
+        ftmoe::set_last_error("ft_slot_acquire: expert id outside [0, table_len)");
+        return FT_ERR_INVALID_ARG;
+      }
+      if (!seen[e]) { seen[e] = 1; want.push_back(e); }
+    }
+  }
+  if ((int)want.size() > m->capacity) {
+    ftmoe::set_last_error("ft_slot_acquire: more distinct experts than slots (cache too small)");
+    return FT_ERR_CAPACITY;
+  }
+  for (int e : want) {
+    const uint64_t key = slot_key(layer, e);
+    if (!m->resident.count(key) && !m->banks.count(key)) {
+      ftmoe::set_last_error("ft_slot_acquire: a missing expert has no registered host bank");
+      return FT_ERR_NOT_RESIDENT;
+    }
+  }
+  // pin: hits move to the front; they are protected from eviction by this call
+  std::unordered_map<uint64_t, char> pinned;
+  for (int e : want) {
+    const uint64_t key = slot_key(layer, e);
+    auto it = m->resident.find(key);
+    pinned[key] = 1;
+    if (it != m->resident.end()) {
+      m->lru.splice(m->lru.begin(), m->lru, it->second.it);
+      ++m->stats.hits;
+    }
+  }
+  std::vector<int32_t> table(table_len, -1);
+  const size_t slot_bytes = size_t(m->layout.slot_bytes);
+  // A slot may still be read by work already enqueued on the compute stream:
+  // fills that reuse an evicted slot wait for that work on the copy stream.
+  bool copy_waits = false;
+  for (int e : want) {
+    const uint64_t key = slot_key(layer, e);
+    auto it = m->resident.find(key);
+    if (it != m->resident.end()) {
+      table[e] = it->second.slot;
+      continue;
+    }
+    int slot;
+    if (!m->free_slots.empty()) {
+      slot = m->free_slots.back();
+      m->free_slots.pop_back();
+    } else {
+      // evict the least recently used entry that this call does not need
+      auto victim = m->lru.end();
+      for (auto r = m->lru.rbegin(); r != m->lru.rend(); ++r)
+        if (!pinned.count(*r)) { victim = std::prev(r.base()); break; }
+      if (victim == m->lru.end()) {
+        ftmoe::set_last_error("ft_slot_acquire: no evictable slot");
+        return FT_ERR_CAPACITY;
+      }
+      slot = m->resident[*victim].slot;
+      m->resident.erase(*victim);
+      m->lru.erase(victim);
+      ++m->stats.evictions;
+      if (!m->host_only && !copy_waits) {
+        if (cudaEventRecord(m->compute_mark, reinterpret_cast<cudaStream_t>(compute)) != cudaSuccess ||
+            cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(copy), m->compute_mark, 0) != cudaSuccess) {
+          m->free_slots.push_back(slot);
+          ftmoe::set_last_error("ft_slot_acquire: ordering the fill after compute failed");
+          return FT_ERR_CUDA;
+        }
+        copy_waits = true;
+      }
+    }
+    cudaError_t err = cudaSuccess;
+    if (m->inject_failures > 0) {
+      --m->inject_failures;
+      err = cudaErrorUnknown;
+    } else if (!m->host_only) {
+      err = cudaMemcpyAsync(m->pool + size_t(slot) * slot_bytes, m->banks[key], slot_bytes,
+                            cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(copy));
+    }
+    if (err != cudaSuccess) {
+      m->free_slots.push_back(slot);   // the slot holds nothing valid now
+      ftmoe::set_last_error("ft_slot_acquire: host-to-device fill failed");
+      return FT_ERR_CUDA;
+    }
+    m->lru.push_front(key);
+    m->resident[key] = ft_slot_mgr::Entry{slot, m->lru.begin()};
+    table[e] = slot;
+    ++m->stats.misses;
+    m->stats.bytes_h2d += int64_t(slot_bytes);
+  }
+  m->host_table = table;
+  if (m->host_only) {   // device_table is host memory in this mode
+    std::memcpy(device_table, table.data(), size_t(table_len) * 4);
+    return FT_OK;
+  }
+  // upload the table from page-locked staging so the copy stays asynchronous
+  if (m->pinned_table_len < table_len) {
+    // the previous upload (if any) must have finished reading the old buffer
+    if (m->pinned_table) {
+      cudaEventSynchronize(m->done);
+      cudaFreeHost(m->pinned_table);
+    }
+    m->pinned_table = nullptr;
+    m->pinned_table_len = 0;
+    if (cudaMallocHost(reinterpret_cast<void**>(&m->pinned_table), size_t(table_len) * 4) != cudaSuccess) {
+      ftmoe::set_last_error("ft_slot_acquire: cudaMallocHost failed");
+      return FT_ERR_CUDA;
+    }
+    m->pinned_table_len = table_len;
+  } else {
+    cudaEventSynchronize(m->done);  // previous upload finished reading the staging buffer
+  }
+  std::memcpy(m->pinned_table, table.data(), size_t(table_len) * 4);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy);
+  if (cudaMemcpyAsync(device_table, m->pinned_table, size_t(table_len) * 4, cudaMemcpyHostToDevice, cs) !=
+          cudaSuccess ||
+      cudaEventRecord(m->done, cs) != cudaSuccess ||
+      cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(compute), m->done, 0) != cudaSuccess) {
+    ftmoe::set_last_error("ft_slot_acquire: table upload failed");
+    return FT_ERR_CUDA;
+  }
+  return FT_OK;
+}
+
+extern "C" int ft_slot_stats(const ft_slot_mgr* m, ft_slot_stats_t* out) {
+  if (!m || !out) return FT_ERR_INVALID_ARG;
+  *out = m->stats;
+  return FT_OK;
+}
+
+extern "C" int ft_slot_destroy(ft_slot_mgr* m) {
+  if (!m) return FT_ERR_INVALID_ARG;
+  if (m->done) {
+    cudaEventSynchronize(m->done);
+    cudaEventDestroy(m->done);
+  }
+  if (m->compute_mark) cudaEventDestroy(m->compute_mark);
+  if (m->pinned_table) cudaFreeHost(m->pinned_table);
+  delete m;
+  return FT_OK;
+}

@@ -1,0 +1,154 @@
+"""Python-side plumbing around the C ABI: device buffers (torch), streams,
+the expert slot pool and the slot manager.
+
+Every step of the layer runs in libftmoe.so; this module only allocates
+memory with torch and forwards pointers (there is no fallback path).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import FT_DOWN, FT_GATE, FT_UP
+
+
+def _ptr(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream(s: Optional[torch.cuda.Stream]) -> int:
+    s = torch.cuda.current_stream() if s is None else s
+    return s.cuda_stream
+
+
+class ExpertPool:
+    """A device pool of NVFP4 expert slots laid out by ft_nvfp4_slot_layout_init."""
+
+    def __init__(self, H: int, I: int, num_slots: int, device="cuda"):
+        self.H, self.I, self.num_slots = H, I, num_slots
+        self.layout = _lib.slot_layout(H, I, num_slots)
+        self.slot_bytes = int(self.layout.slot_bytes)
+        self.buf = torch.zeros(num_slots * self.slot_bytes, dtype=torch.uint8, device=device)
+        self._pack_ws = torch.zeros(256, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    def shape(self, mat: int):
+        return (self.I, self.H) if mat in (FT_GATE, FT_UP) else (self.H, self.I)
+
+    def pack_into(self, slot: int, mat: int, w: torch.Tensor, stream=None) -> None:
+        """Quantise fp32 weights w [N, K] (on the device) into `slot`."""
+        N, K = self.shape(mat)
+        assert w.shape == (N, K) and w.dtype == torch.float32 and w.is_cuda and w.is_contiguous()
+        L = self.layout
+        base = self.ptr + slot * self.slot_bytes
+        _lib.nvfp4_pack(w.data_ptr(), N, K, base + L.codes_off[mat], base + L.scales_off[mat],
+                        L.ld_scale[mat], base + L.global_off[mat], self._pack_ws.data_ptr(), _stream(stream))
+
+    def slot_view(self, slot: int) -> torch.Tensor:
+        return self.buf[slot * self.slot_bytes:(slot + 1) * self.slot_bytes]
+
+    def tensor_bytes(self, slot: int, mat: int):
+        """(codes uint8 [N, K/2], scales uint8 [N, ld], global fp32) of one tensor, on the host."""
+        N, K = self.shape(mat)
+        L = self.layout
+        s = self.slot_view(slot)
+        codes = s[L.codes_off[mat]:L.codes_off[mat] + N * K // 2].view(N, K // 2).cpu().numpy()
+        scales = s[L.scales_off[mat]:L.scales_off[mat] + N * L.ld_scale[mat]].view(N, L.ld_scale[mat]).cpu().numpy()
+        g = s[L.global_off[mat]:L.global_off[mat] + 4].cpu().numpy().view("float32")[0]
+        return codes, scales, float(g)
+
+
+class MoELayer:
+    """Buffers and calls for one MoE FFN layer of fixed (T, E, k, H, I)."""
+
+    def __init__(self, T: int, E: int, k: int, H: int, I: int, mode: int = _lib.FT_ROUTE_SOFTMAX_RENORM,
+                 device="cuda"):
+        self.T, self.E, self.k, self.H, self.I, self.mode = T, E, k, H, I, mode
+        P = T * k
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.ids = torch.empty((T, k), **i32)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.offsets = torch.empty(E + 1, **i32)
+        self.perm_src = torch.empty(P, **i32)
+        self.pair_to_row = torch.empty(P, **i32)
+        self.out_perm = torch.empty((P, H), dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.perm_ws_bytes = _lib.permute_workspace_size(T, k, E)
+        self.perm_ws = torch.empty(max(self.perm_ws_bytes, 256), dtype=torch.uint8, device=dev)
+        self.ffn_ws_bytes = _lib.ffn_workspace_size(T, H, I, E, k)
+        self.ffn_ws = torch.empty(max(self.ffn_ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    def route(self, logits: torch.Tensor, stream=None) -> None:
+        _lib.route(logits.data_ptr(), self.T, self.E, self.k, self.mode, self.ids.data_ptr(), self.w.data_ptr(),
+                   _stream(stream))
+
+    def permute(self, stream=None) -> None:
+        _lib.permute(self.ids.data_ptr(), self.T, self.k, self.E, self.offsets.data_ptr(), self.perm_src.data_ptr(),
+                     self.pair_to_row.data_ptr(), self.perm_ws.data_ptr(), self.perm_ws_bytes, _stream(stream))
+
+    def ffn(self, x: torch.Tensor, slot_table: torch.Tensor, pool: ExpertPool, stream=None) -> None:
+        _lib.ffn_nvfp4(x.data_ptr(), self.T, self.H, self.I, self.E, self.k, self.perm_src.data_ptr(),
+                       self.offsets.data_ptr(), slot_table.data_ptr(), pool.ptr, pool.layout,
+                       self.out_perm.data_ptr(), self.ffn_ws.data_ptr(), self.ffn_ws_bytes, _stream(stream))
+
+    def combine(self, stream=None) -> None:
+        _lib.combine(self.out_perm.data_ptr(), self.pair_to_row.data_ptr(), self.w.data_ptr(), self.T, self.k,
+                     self.H, self.y.data_ptr(), _stream(stream))
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, slot_table: torch.Tensor, pool: ExpertPool,
+                stream=None) -> torch.Tensor:
+        """route -> permute -> ffn -> combine, enqueued on one stream."""
+        assert x.dtype == torch.bfloat16 and x.shape == (self.T, self.H) and x.is_contiguous()
+        assert logits.dtype == torch.float32 and logits.shape == (self.T, self.E) and logits.is_contiguous()
+        assert slot_table.dtype == torch.int32 and slot_table.numel() == self.E
+        self.route(logits, stream)
+        self.permute(stream)
+        self.ffn(x, slot_table, pool, stream)
+        self.combine(stream)
+        return self.y
+
+
+class SlotManager:
+    """ctypes wrapper of the host LRU slot manager (ft_slot_*)."""
+
+    def __init__(self, capacity: int, layout: _lib.SlotLayout, pool_ptr: int = 0, host_only: bool = False):
+        h = ctypes.c_void_p()
+        flags = _lib.FT_SLOT_HOST_ONLY if host_only else _lib.FT_SLOT_DEVICE
+        _lib.check(_lib.lib().ft_slot_create(ctypes.byref(h), capacity, ctypes.byref(layout),
+                                             ctypes.c_void_p(pool_ptr or None), flags))
+        self.h = h
+        self.layout = layout
+
+    def register_host(self, layer: int, expert: int, src_ptr: int) -> None:
+        _lib.check(_lib.lib().ft_slot_register_host(self.h, layer, expert, ctypes.c_void_p(src_ptr)))
+
+    def acquire(self, layer: int, ids, table_ptr: int, table_len: int, compute=0, copy=0) -> None:
+        arr = (ctypes.c_int32 * len(ids))(*[int(i) for i in ids])
+        _lib.check(_lib.lib().ft_slot_acquire(self.h, layer, arr, len(ids), ctypes.c_void_p(table_ptr), table_len,
+                                              ctypes.c_void_p(compute or None), ctypes.c_void_p(copy or None)))
+
+    def inject_copy_failures(self, n: int) -> None:
+        _lib.check(_lib.lib().ft_slot_inject_copy_failures(self.h, n))
+
+    def stats(self) -> dict:
+        s = _lib.SlotStats()
+        _lib.check(_lib.lib().ft_slot_stats(self.h, ctypes.byref(s)))
+        return {"hits": s.hits, "misses": s.misses, "evictions": s.evictions, "bytes_h2d": s.bytes_h2d}
+
+    def close(self) -> None:
+        if self.h:
+            _lib.lib().ft_slot_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

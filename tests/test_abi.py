@@ -1,0 +1,100 @@
+"""The C-ABI library loads, exports every function include/ftmoe.h declares,
+and rejects bad arguments before touching the GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from moe_expert_layer_renorm_b200 import _lib
+from moe_expert_layer_renorm_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ftmoe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*FT_API\s+(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(ft_[a-z0-9_]+)\s*\(", src,
+                       flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for required in ("ft_moe_route", "ft_moe_permute", "ft_moe_ffn_nvfp4", "ft_moe_combine", "ft_nvfp4_pack",
+                     "ft_slot_create", "ft_slot_acquire", "ft_slot_destroy", "ft_last_error"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_ctypes_signatures_cover_the_header():
+    assert set(declared_functions()) <= set(_lib._SIGS)
+
+
+def test_version(L):
+    assert "sm_100a" in _lib.version()
+
+
+def test_slot_layout_rules(L):
+    for H, I in ((256, 512), (2048, 768), (2048, 512), (2880, 2880), (320, 448)):
+        lay = _lib.slot_layout(H, I, 7)
+        rows = (I, I, H)
+        ks = (H, H, I)
+        ends = []
+        for m in range(3):
+            assert lay.ld_scale[m] % 16 == 0 and lay.ld_scale[m] >= ks[m] // 16
+            assert lay.codes_off[m] % 256 == 0 and lay.scales_off[m] % 256 == 0
+            assert lay.codes_off[m] + rows[m] * ks[m] // 2 <= lay.scales_off[m]
+            ends.append(lay.scales_off[m] + rows[m] * lay.ld_scale[m])
+        assert lay.codes_off[1] >= ends[0] and lay.codes_off[2] >= ends[1]
+        assert min(lay.global_off) >= ends[2]
+        assert lay.slot_bytes % 256 == 0 and lay.slot_bytes >= max(lay.global_off) + 4
+        assert lay.num_slots == 7
+    # 2880/16 = 180 scale bytes per row, padded to 192 for 16-byte TMA rows
+    assert _lib.slot_layout(2880, 2880, 1).ld_scale[0] == 192
+
+
+def test_slot_layout_rejects_bad_sizes(L):
+    with pytest.raises(_lib.FtError) as ei:
+        _lib.slot_layout(100, 512, 1)
+    assert ei.value.code == _lib.FT_ERR_INVALID_ARG
+
+
+def test_argument_checks_need_no_gpu(L):
+    # k > E
+    assert L.ft_moe_route(None, 4, 8, 9, 0, None, None, None) == _lib.FT_ERR_INVALID_ARG
+    assert b"k <=" in L.ft_last_error()
+    # E > 1024
+    assert L.ft_moe_route(None, 4, 2000, 2, 0, None, None, None) == _lib.FT_ERR_INVALID_ARG
+    # T == 0 is a no-op
+    assert L.ft_moe_route(None, 0, 8, 2, 0, None, None, None) == _lib.FT_OK
+    assert L.ft_moe_combine(None, None, None, 0, 2, 256, None, None) == _lib.FT_OK
+    assert L.ft_moe_combine(None, None, None, 4, 2, 250, None, None) == _lib.FT_ERR_INVALID_ARG
+    lay = _lib.slot_layout(256, 512, 8)
+    # unsupported sizes
+    assert L.ft_moe_ffn_nvfp4(None, 4, 192, 512, 8, 2, None, None, None, None, ctypes.byref(lay), None, None, 0,
+                              None) == _lib.FT_ERR_UNSUPPORTED
+    # null pointers
+    assert L.ft_moe_ffn_nvfp4(None, 4, 256, 512, 8, 2, None, None, None, None, ctypes.byref(lay), None, None, 0,
+                              None) == _lib.FT_ERR_INVALID_ARG
+    assert L.ft_nvfp4_pack(None, 4, 20, None, None, 2, None, None, None) == _lib.FT_ERR_INVALID_ARG
+
+
+def test_workspace_queries(L):
+    assert _lib.permute_workspace_size(16, 2, 8) == 0            # one chunk: no workspace
+    assert _lib.permute_workspace_size(8192, 10, 512) == 80 * 512 * 4
+    small = _lib.ffn_workspace_size(16, 256, 512, 8, 2)
+    big = _lib.ffn_workspace_size(4096, 2048, 768, 128, 8)
+    assert small > 16 * 2 * 512 * 2 and big > 4096 * 8 * 768 * 2
+    assert _lib.ffn_workspace_size(0, 2048, 768, 128, 8) == 0
