@@ -138,16 +138,19 @@ FT_API size_t ft_moe_permute_workspace_size(int T, int k, int E);
  * t = perm_src[r] / k), with the expert's tensors at
  * slot_pool + slot_table[e] * layout->slot_bytes:
  *   h[r]        = silu(gG * (Qg x_t)) * (gU * (Qu x_t))        (I values)
- *   out_perm[r] = bf16(gD * (Qd h[r]))                          (H values)
+ *   out_perm[r] = gD * (Qd h[r])                                (H values, fp32)
  * where Q* are the E2M1*E4M3 dequantised weights (exact in bf16), g* the
  * fp32 global scales, products accumulate in fp32 on the tensor cores, and
- * h is rounded to bf16 before the down projection.
+ * h is rounded to bf16 before the down projection (it is that MMA's
+ * operand).  The expert outputs stay fp32 so that the layer output meets
+ * |y - y_exact| <= 1e-2 rms(y) + 1e-3: a bf16 rounding of them (or of y) alone
+ * would already reach that bound at the tails of the output distribution.
  *   x              device bf16 [T, H]
  *   perm_src       device int32 [T*k]     from ft_moe_permute
  *   expert_offsets device int32 [E+1]     from ft_moe_permute
  *   slot_table     device int32 [E]       expert -> slot; -1 = not resident
  *   slot_pool      device, layout->num_slots * layout->slot_bytes bytes, 256-B aligned
- *   out_perm       device bf16 [T*k, H]   (out)
+ *   out_perm       device fp32 [T*k, H]   (out)
  *   ws             device workspace of ft_moe_ffn_workspace_size bytes, 256-B aligned
  * A non-empty group whose slot is -1 sets FT_DEV_NOT_RESIDENT and its rows are
  * left unwritten.  H and I must be multiples of 64 and match the layout.
@@ -160,10 +163,11 @@ FT_API int ft_moe_ffn_nvfp4(const void* x, int T, int H, int I, int E, int k,
 FT_API size_t ft_moe_ffn_workspace_size(int T, int H, int I, int E, int k);
 
 /*
- * Combine: y[t, :] = bf16( sum_{j<k} topk_w[t,j] * out_perm[pair_to_row[t*k+j], :] ),
+ * Combine: y[t, :] = sum_{j<k} topk_w[t,j] * out_perm[pair_to_row[t*k+j], :],
  * summed in fp32 in the order j = 0..k-1.
- *   out_perm device bf16 [T*k, H], pair_to_row device int32 [T*k],
- *   topk_w device fp32 [T, k], y device bf16 [T, H] (out).  H % 8 == 0.
+ *   out_perm device fp32 [T*k, H], pair_to_row device int32 [T*k],
+ *   topk_w device fp32 [T, k], y device fp32 [T, H] (out).  H % 4 == 0;
+ *   out_perm and y 16-byte aligned.
  */
 FT_API int ft_moe_combine(const void* out_perm, const int32_t* pair_to_row, const float* topk_w,
                    int T, int k, int H, void* y, ft_stream_t stream);
@@ -190,6 +194,17 @@ FT_API int ft_nvfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* 
  * device.  Synchronises the device.  *status receives an FT_DEV_* code.
  */
 FT_API int ft_device_status(int* status, int clear);
+
+/*
+ * Where the first recorded device status came from (synchronises the
+ * device): detail[0] code, [1] block, [2] warp, [3] barrier kind (for a wait
+ * timeout: 1 weight-stage free, 2 weight-stage full, 3 token-stage free,
+ * 4 token-stage full, 5 operand-slot free, 6 operand-slot full,
+ * 7 accumulator free, 8 accumulator full), [4] the waiting role's counter,
+ * [5] work unit, [6] microseconds waited, [7] reserved.  Cleared together
+ * with the status word by ft_device_status(..., clear = 1).
+ */
+FT_API int ft_device_status_detail(int64_t detail[8]);
 
 /* ---------------------------------------------------------------------------
  * Expert slot manager: a host-side LRU over (layer, expert) keys, mirroring

@@ -74,6 +74,7 @@ _SIGS = {
     "ft_moe_combine": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
     "ft_nvfp4_pack": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "ft_device_status": (c_int, [POINTER(c_int), c_int]),
+    "ft_device_status_detail": (c_int, [POINTER(c_int64)]),
     "ft_slot_create": (c_int, [POINTER(c_void_p), c_int, POINTER(SlotLayout), c_void_p, c_int]),
     "ft_slot_register_host": (c_int, [c_void_p, c_int, c_int, c_void_p]),
     "ft_slot_acquire": (c_int, [c_void_p, c_int, POINTER(c_int32), c_int, c_void_p, c_int, c_void_p, c_void_p]),
@@ -149,6 +150,12 @@ def device_status(clear: bool = True) -> int:
     v = c_int(0)
     check(lib().ft_device_status(ctypes.byref(v), 1 if clear else 0))
     return v.value
+
+
+def device_status_detail() -> list:
+    d = (c_int64 * 8)()
+    check(lib().ft_device_status_detail(d))
+    return [int(v) for v in d]
 
 
 def profile_enable(on: bool) -> None:

@@ -126,8 +126,8 @@ extern "C" int ft_moe_ffn_nvfp4(const void* x, int T, int H, int I, int E, int k
 
 extern "C" int ft_moe_combine(const void* out_perm, const int32_t* pair_to_row, const float* w, int T, int k,
                               int H, void* y, ft_stream_t stream) {
-  if (T < 0 || k < 1 || k > 1024 || H < 8 || H % 8)
-    return fail(FT_ERR_INVALID_ARG, "ft_moe_combine: need k >= 1 and H a positive multiple of 8");
+  if (T < 0 || k < 1 || k > 1024 || H < 4 || H % 4)
+    return fail(FT_ERR_INVALID_ARG, "ft_moe_combine: need k >= 1 and H a positive multiple of 4");
   if (T == 0) return FT_OK;
   if (!out_perm || !pair_to_row || !w || !y) return fail(FT_ERR_INVALID_ARG, "ft_moe_combine: null pointer");
   if ((reinterpret_cast<uintptr_t>(out_perm) & 15) || (reinterpret_cast<uintptr_t>(y) & 15))
@@ -156,11 +156,20 @@ extern "C" int ft_device_status(int* status, int clear) {
   if (e != cudaSuccess) return cuda_fail(e, "ft_device_status");
   if (clear) {
     const int zero = 0;
-    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+    const long long zeros[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    e = cudaMemcpyToSymbol(g_device_status_detail, zeros, sizeof(zeros));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(e, "ft_device_status");
   }
   *status = v;
   return FT_OK;
+}
+
+extern "C" int ft_device_status_detail(int64_t* detail) {
+  if (!detail) return fail(FT_ERR_INVALID_ARG, "ft_device_status_detail: null pointer");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(detail, g_device_status_detail, 8 * sizeof(long long));
+  return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_device_status_detail");
 }
 
 extern "C" int ft_profile_enable(int on) {

@@ -8,13 +8,15 @@
 // Data path of one CTA (persistent; 16 warps):
 //   warp 0      TMA: packed E2M1 codes (128 rows x 128 B, 128-byte swizzle)
 //               and E4M3 scales (128 rows x 16 B) of each matrix, 256 K per stage
-//   warps 2-3   cp.async: the unit's token rows (bf16, 64 K per chunk) into
+//   warp 2      TMA: the unit's token rows (bf16, 64 K per chunk) into
 //               128-byte-swizzled K-major shared memory (the MMA's B operand);
-//               GEMM1 gathers x rows through perm_src, GEMM2 reads h rows
+//               GEMM1 gathers x rows through perm_src four at a time
+//               (tile::gather4), GEMM2 loads 16-row tiles of h
 //   warps 4-11  dequantise one 64-K chunk per step: E2M1 -> f16 (cvt) times the
 //               E4M3 block scale (exact in f16), widened to bf16 (exact), and
 //               stored with tcgen05.st straight into tensor memory, where the
 //               MMA reads it as its A operand (no shared-memory round trip)
+//   warp 3      idle
 //   warp 1      one thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
 //               accumulators in tensor memory) and commits to the barriers
 //   warps 12-15 epilogue: tcgen05.ld of the accumulators, fp32 global scale,
@@ -41,8 +43,7 @@ constexpr int kMatStageBytes = kCodesBytes + kScaleBytes;   // 18 KB, multiple o
 constexpr int kThreads = 512;
 
 struct FfnParams {
-  const __nv_bfloat16* act;   // GEMM1: x [T, K]; GEMM2: h [P, K]
-  const int32_t* perm_src;    // GEMM1: row -> pair (token = pair / k_top); GEMM2: null
+  const int32_t* perm_src;    // GEMM1: row -> pair (token = pair / k_top); GEMM2: null (row -> row)
   int k_top;
   int K;                      // reduction length
   int M;                      // output features (rows of the weight matrices)
@@ -56,7 +57,7 @@ struct FfnParams {
   const uint8_t* pool;
   long long slot_bytes;
   long long global_off[2];
-  __nv_bfloat16* out;         // GEMM1: h [P, M]; GEMM2: out_perm [P, M]
+  void* out;                  // GEMM1: h bf16 [P, M]; GEMM2: out_perm fp32 [P, M]
   float* partials;            // split-K partial accumulators
   int* counters;              // split-K arrival counters, 4 per (tile, m_tile): one per epilogue warp
 };
@@ -124,9 +125,13 @@ __device__ __forceinline__ void dequant_chunk(const uint4& c0, const uint4& c1, 
 
 // ---------------------------------------------------------- pipeline ---
 
+// Barrier kinds, recorded with a wait timeout.
+enum : int { kTagWEmpty = 1, kTagWFull, kTagBEmpty, kTagBFull, kTagAEmpty, kTagAFull, kTagDEmpty, kTagDFull };
+
 struct Abort {
   volatile int* flag;
-  __device__ bool wait(uint64_t* bar, uint32_t parity) const {
+  __device__ bool wait(uint64_t* bar, uint32_t parity, int tag = 0, long long counter = 0,
+                       long long unit = 0) const {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     uint32_t n = 0;
@@ -134,8 +139,9 @@ struct Abort {
       if (mbar_try_wait(bar, parity)) return true;
       if ((++n & 63u) == 0) {
         if (*flag) return false;
-        if (globaltimer_ns() - t0 > 1000000000ull) {
-          set_device_status(FT_DEV_WAIT_TIMEOUT);
+        const uint64_t dt = globaltimer_ns() - t0;
+        if (dt > 1000000000ull) {
+          set_device_status_detail(FT_DEV_WAIT_TIMEOUT, tag, counter, unit, (long long)(dt / 1000));
           *flag = 1;
           return false;
         }
@@ -146,11 +152,19 @@ struct Abort {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// GEMM1 stores h in bf16 (it is the next MMA's operand); GEMM2 stores the
+// expert outputs in fp32 so that only the combine's own fp32 sum rounds them.
+template <int NMAT>
+__device__ __forceinline__ void store_out(void* out, size_t idx, float v) {
+  if (NMAT == 2) static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
+  else static_cast<float*>(out)[idx] = v;
+}
+
 template <int NMAT, int BN, int WS, int BS, int AS, int DB>
 __global__ void __launch_bounds__(kThreads, 1)
 ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0,
                 const __grid_constant__ CUtensorMap tm_scales0, const __grid_constant__ CUtensorMap tm_codes1,
-                const __grid_constant__ CUtensorMap tm_scales1) {
+                const __grid_constant__ CUtensorMap tm_scales1, const __grid_constant__ CUtensorMap tm_act) {
   using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -173,7 +187,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < WS; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], 8); }
-    for (int i = 0; i < BS; ++i) { mbar_init(&b_full[i], 64); mbar_init(&b_empty[i], 1); }
+    for (int i = 0; i < BS; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
     for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < DB; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4); }
     mbar_init(drain_bar, 1);
@@ -184,6 +198,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
     prefetch_tmap(&tm_codes0); prefetch_tmap(&tm_scales0);
     if (NMAT > 1) { prefetch_tmap(&tm_codes1); prefetch_tmap(&tm_scales1); }
   }
+  if (warp == 2 && lane == 0) prefetch_tmap(&tm_act);
   if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -216,7 +231,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
         const int slot = __ldg(p.slot_table + e);
         for (int ws = ws0; ws < ws1; ++ws, ++wi) {
           const int s = wi % WS;
-          if (!(ok = ab.wait(&w_empty[s], ((wi / WS) & 1) ^ 1))) break;
+          if (!(ok = ab.wait(&w_empty[s], ((wi / WS) & 1) ^ 1, kTagWEmpty, wi, u))) break;
           mbar_arrive_expect_tx(&w_full[s], NMAT * kMatStageBytes);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
@@ -241,14 +256,14 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
         int e, mt, rb, nr, ws0, ws1, kc0, kc1;
         unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
         const int ds = di % DB;
-        if (!(ok = ab.wait(&d_empty[ds], ((di / DB) & 1) ^ 1))) break;
+        if (!(ok = ab.wait(&d_empty[ds], ((di / DB) & 1) ^ 1, kTagDEmpty, di, u))) break;
         tc_fence_after();
         const int n_eff = (nr + 15) & ~15;
         const uint32_t idesc = make_idesc_f16(128, n_eff);
         for (int c = kc0; c < kc1; ++c, ++q) {
           const int as = q % AS, bs = q % BS;
-          if (!(ok = ab.wait(&a_full[as], (q / AS) & 1))) break;
-          if (!(ok = ab.wait(&b_full[bs], (q / BS) & 1))) break;
+          if (!(ok = ab.wait(&a_full[as], (q / AS) & 1, kTagAFull, q, u))) break;
+          if (!(ok = ab.wait(&b_full[bs], (q / BS) & 1, kTagBFull, q, u))) break;
           tc_fence_after();
           const uint32_t b_addr = smem_u32(b_smem + bs * Cfg::kBStageBytes);
 #pragma unroll
@@ -274,54 +289,53 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
         while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
       }
     }
-  } else if (warp < 4) {
-    // --------------------------------------------- B (token) loader ---
-    // Thread tb copies 16-byte column c16 = tb % 8 of rows n = tb / 8 + 8 i.
-    // Up to BS - 1 chunks stay in flight; a chunk's barrier is signalled once
-    // this thread's copies for it have landed.
-    const int tb = threadIdx.x - 64;  // 0..63
-    const int c16 = tb & 7, n_first = tb >> 3;
-    constexpr int kRowsPerThread = BN / 8;
-    constexpr int kLag = BS - 1;
-    uint32_t q = 0, pending = 0;
+  } else if (warp == 2) {
+    // --------------------------------------------- B (token) producer ---
+    // The lanes look up the unit's token rows; lane 0 issues one TMA per
+    // 4 rows (GEMM1, gathered x rows) or per 16 rows (GEMM2, contiguous h
+    // rows) for every 64-K chunk.  Rows past the group end but below the
+    // MMA's N repeat the last real row (their results are never stored).
+    uint32_t q = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       int e, mt, rb, nr, ws0, ws1, kc0, kc1;
       unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
-      int rows[kRowsPerThread];
-#pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) {
-        const int n = n_first + 8 * i;
-        rows[i] = n < nr ? (p.perm_src ? __ldg(p.perm_src + rb + n) / p.k_top : rb + n) : -1;
-      }
       const int n_eff = (nr + 15) & ~15;
-      for (int c = kc0; c < kc1; ++c, ++q) {
-        const int bs = q % BS;
-        if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&b_empty[bs], ((q / BS) & 1) ^ 1)))) break;
-        const uint32_t dst0 = smem_u32(b_smem + bs * Cfg::kBStageBytes);
-        const int kk = c * kKC + c16 * 8;
-#pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          const int n = n_first + 8 * i;
-          if (n < n_eff) {
-            const bool live = rows[i] >= 0 && kk < p.K;
-            const __nv_bfloat16* src = live ? p.act + size_t(rows[i]) * p.K + kk : p.act;
-            cp_async_16(dst0 + n * 128 + ((c16 ^ (n & 7)) << 4), src, live ? 16u : 0u);
+      for (int n = lane; n < n_eff; n += 32) {
+        const int r = rb + min(n, nr - 1);
+        rowidx[n] = p.perm_src ? __ldg(p.perm_src + r) / p.k_top : r;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        for (int c = kc0; c < kc1; ++c, ++q) {
+          const int bs = q % BS;
+          if (!(ok = ab.wait(&b_empty[bs], ((q / BS) & 1) ^ 1, kTagBEmpty, q, u))) break;
+          mbar_arrive_expect_tx(&b_full[bs], uint32_t(n_eff) * 128u);
+          uint8_t* dst = b_smem + bs * Cfg::kBStageBytes;
+          const int k0 = c * kKC;
+          if (p.perm_src) {
+            for (int n = 0; n < n_eff; n += 4)
+              tma_gather4(dst + n * 128, &tm_act, &b_full[bs], k0, rowidx[n], rowidx[n + 1], rowidx[n + 2],
+                          rowidx[n + 3]);
+          } else {
+            for (int n = 0; n < n_eff; n += 16) tma_load_2d(dst + n * 128, &tm_act, &b_full[bs], k0, rb + n);
           }
         }
-        cp_async_commit();
-        if (++pending > kLag) {
-          cp_async_wait<kLag>();
-          fence_proxy_async_smem();
-          mbar_arrive(&b_full[(q - kLag) % BS]);
-          --pending;
-        }
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      q = __shfl_sync(0xFFFFFFFFu, q, 0);
+      __syncwarp();
+    }
+    if (lane == 0) {   // drain: the last copy into every B stage has landed
+      for (uint32_t j = (q > BS ? q - BS : 0); j < q; ++j) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&b_full[j % BS], (j / BS) & 1) && globaltimer_ns() - t0 < 1000000000ull) {}
       }
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    for (; pending > 0; --pending) mbar_arrive(&b_full[(q - pending) % BS]);
-  } else if (warp < 12) {
+  } else if (warp == 3) {
+    // idle: keeps the dequantising warps at warp indices 4..11, so that warp % 4
+    // names the 32-lane quarter of tensor memory each of them may access
+  } else if (warp >= 4 && warp < 12) {
     // -------------------------------------------------- dequantise ---
     const int g = (warp - 4) >> 2;            // warpgroup: even / odd chunks
     const int quarter = warp & 3;
@@ -334,12 +348,12 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
       unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
       for (int ws = ws0; ws < ws1 && ok; ++ws, ++wi) {
         const int s = wi % WS;
-        if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&w_full[s], (wi / WS) & 1)))) break;
+        if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&w_full[s], (wi / WS) & 1, kTagWFull, wi, u)))) break;
         const int c_end = min(kc1, (ws + 1) * kCPW);
         for (int c = ws * kCPW; c < c_end; ++c, ++q) {
           if ((q & 1) != uint32_t(g)) continue;
           const int as = q % AS;
-          if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&a_empty[as], ((q / AS) & 1) ^ 1)))) break;
+          if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&a_empty[as], ((q / AS) & 1) ^ 1, kTagAEmpty, q, u)))) break;
           tc_fence_after();
           const int cc = c - ws * kCPW;
 #pragma unroll
@@ -362,7 +376,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
         if (lane == 0) mbar_arrive(&w_empty[s]);
       }
     }
-  } else {
+  } else if (warp >= 12 && warp < 16) {
     // ---------------------------------------------------- epilogue ---
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -379,7 +393,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
       float gsc[NMAT];
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) gsc[m] = __ldg(reinterpret_cast<const float*>(sbase + p.global_off[m]));
-      if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&d_full[ds], (di / DB) & 1)))) break;
+      if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&d_full[ds], (di / DB) & 1, kTagDFull, di, u)))) break;
       tc_fence_after();
       const int n_eff = (nr + 15) & ~15;
       const bool split = p.splits > 1;
@@ -400,7 +414,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
             float r;
             if (NMAT == 2) r = silu_mul(gsc[0] * __uint_as_float(v[0][i]), gsc[NMAT - 1] * __uint_as_float(v[NMAT - 1][i]));
             else r = gsc[0] * __uint_as_float(v[0][i]);
-            p.out[size_t(rb + n) * p.M + feat] = __float2bfloat16_rn(r);
+            store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
           }
         }
       }
@@ -431,7 +445,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
               float r;
               if (NMAT == 2) r = silu_mul(gsc[0] * acc[0], gsc[NMAT - 1] * acc[NMAT - 1]);
               else r = gsc[0] * acc[0];
-              p.out[size_t(rb + n) * p.M + feat] = __float2bfloat16_rn(r);
+              store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
             }
           }
           if (lane == 0) p.counters[(u / p.splits) * 4 + quarter] = 0;
@@ -528,8 +542,8 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   pl.nkc1 = H / kKC;
   pl.nkc2 = I / kKC;
   if (pl.decode) {
-    pl.g1 = {32, 1, 0, 5, 4, 4, 2};
-    pl.g2 = {32, 1, 0, 8, 4, 4, 2};
+    pl.g1 = {32, 1, 0, 5, 8, 4, 2};
+    pl.g2 = {32, 1, 0, 8, 8, 4, 2};
   } else {
     pl.g1 = {128, 1, 0, 3, 4, 4, 1};
     pl.g2 = {128, 1, 0, 3, 6, 4, 2};
@@ -598,9 +612,25 @@ static bool make_weight_maps(const uint8_t* pool, const ft_nvfp4_slot_layout& L,
   return true;
 }
 
+// Activation rows (bf16 [rows, K]) as the MMA's B operand, 64-column (128-byte)
+// boxes with the 128-byte swizzle: one-row boxes for tile::gather4, or
+// 16-row boxes for contiguous rows.
+static bool make_act_map(const void* base, int rows, int K, int box_rows, CUtensorMap* m) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+  const cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int NMAT, int BN, int WS, int BS, int AS, int DB>
 static cudaError_t launch_gemm(const FfnParams& p, int grid, const CUtensorMap& c0, const CUtensorMap& s0,
-                               const CUtensorMap& c1, const CUtensorMap& s1, cudaStream_t s) {
+                               const CUtensorMap& c1, const CUtensorMap& s1, const CUtensorMap& act,
+                               cudaStream_t s) {
   ProfileScope prof(NMAT == 2 ? FT_KERNEL_GEMM_GATE_UP : FT_KERNEL_GEMM_DOWN, s);
   using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB>;
   auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB>;
@@ -610,7 +640,7 @@ static cudaError_t launch_gemm(const FfnParams& p, int grid, const CUtensorMap& 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, kThreads, Cfg::kSmemBytes, s>>>(p, c0, s0, c1, s1);
+  kern<<<grid, kThreads, Cfg::kSmemBytes, s>>>(p, c0, s0, c1, s1, act);
   return cudaGetLastError();
 }
 
@@ -650,8 +680,12 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
 
+  CUtensorMap tm_x, tm_h;
+  if (!make_act_map(x, T, H, 1, &tm_x) || !make_act_map(h, T * k, I, 16, &tm_h)) {
+    *why = "cuTensorMapEncodeTiled failed for the activations";
+    return cudaErrorInvalidValue;
+  }
   FfnParams p1{};
-  p1.act = static_cast<const __nv_bfloat16*>(x);
   p1.perm_src = perm_src;
   p1.k_top = k;
   p1.K = H;
@@ -673,7 +707,6 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   const int grid1 = int(std::min<long long>(num_sms, pl.max_units1));
 
   FfnParams p2 = p1;
-  p2.act = h;
   p2.perm_src = nullptr;
   p2.K = I;
   p2.M = H;
@@ -685,17 +718,17 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   p2.num_units = counts + 1;
   p2.global_off[0] = L.global_off[FT_DOWN];
   p2.global_off[1] = L.global_off[FT_DOWN];
-  p2.out = static_cast<__nv_bfloat16*>(out_perm);
+  p2.out = out_perm;
   p2.partials = reinterpret_cast<float*>(w + pl.off_part2);
   p2.counters = cnt2;
   const int grid2 = int(std::min<long long>(num_sms, pl.max_units2));
 
   if (pl.decode) {
-    err = launch_gemm<2, 32, 5, 4, 4, 2>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], s);
-    if (err == cudaSuccess) err = launch_gemm<1, 32, 8, 4, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], s);
+    err = launch_gemm<2, 32, 5, 8, 4, 2>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    if (err == cudaSuccess) err = launch_gemm<1, 32, 8, 8, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   } else {
-    err = launch_gemm<2, 128, 3, 4, 4, 1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], s);
-    if (err == cudaSuccess) err = launch_gemm<1, 128, 3, 6, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], s);
+    err = launch_gemm<2, 128, 3, 4, 4, 1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    if (err == cudaSuccess) err = launch_gemm<1, 128, 3, 6, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   }
   return err;
 }

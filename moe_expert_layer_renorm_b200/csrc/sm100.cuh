@@ -14,6 +14,8 @@ namespace ftmoe {
 // Device status word (error codes are FT_DEV_* below).  The library is built
 // as one translation unit, so this header is included exactly once.
 __device__ int g_device_status = 0;
+// Detail of the first recorded status: {code, block, warp, tag, counter, unit, elapsed_us, 0}.
+__device__ long long g_device_status_detail[8];
 
 enum : int {
   FT_DEV_OK = 0,
@@ -24,6 +26,21 @@ enum : int {
 
 __device__ __forceinline__ void set_device_status(int code) {
   atomicCAS(&g_device_status, 0, code);
+}
+
+// Record `code` with where it happened; only the first caller's detail is kept.
+__device__ __forceinline__ void set_device_status_detail(int code, int tag, long long counter, long long unit,
+                                                         long long elapsed_us) {
+  if (atomicCAS(&g_device_status, 0, code) == 0) {
+    g_device_status_detail[0] = code;
+    g_device_status_detail[1] = blockIdx.x;
+    g_device_status_detail[2] = threadIdx.x >> 5;
+    g_device_status_detail[3] = tag;
+    g_device_status_detail[4] = counter;
+    g_device_status_detail[5] = unit;
+    g_device_status_detail[6] = elapsed_us;
+    __threadfence();
+  }
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -88,6 +105,27 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];"
       ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// 2-D tiled TMA load (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// TMA row gather (no multicast): four rows y0..y3 of a 2-D tensor whose map
+// has a one-row box, columns [x, x + box width), written as four consecutive
+// rows of the destination tile.
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const void* tmap, uint64_t* bar, int x, int y0,
+                                            int y1, int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+      ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
       : "memory");
 }
 

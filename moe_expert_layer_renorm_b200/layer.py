@@ -78,8 +78,8 @@ class MoELayer:
         self.offsets = torch.empty(E + 1, **i32)
         self.perm_src = torch.empty(P, **i32)
         self.pair_to_row = torch.empty(P, **i32)
-        self.out_perm = torch.empty((P, H), dtype=torch.bfloat16, device=dev)
-        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.out_perm = torch.empty((P, H), dtype=torch.float32, device=dev)
+        self.y = torch.empty((T, H), dtype=torch.float32, device=dev)
         self.perm_ws_bytes = _lib.permute_workspace_size(T, k, E)
         self.perm_ws = torch.empty(max(self.perm_ws_bytes, 256), dtype=torch.uint8, device=dev)
         self.ffn_ws_bytes = _lib.ffn_workspace_size(T, H, I, E, k)

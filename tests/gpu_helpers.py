@@ -54,7 +54,7 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
 
 
 def run_gpu(w: inputs.Workload, T: Optional[int] = None, layer: int = 0, pool=None, slot_table=None,
-            li: Optional[inputs.LayerInputs] = None) -> GpuRun:
+            li: Optional[inputs.LayerInputs] = None, expect_status: int = 0) -> GpuRun:
     li = li or inputs.make_layer_inputs(w, layer, T)
     T = li.x_bits.shape[0]
     if pool is None:
@@ -63,8 +63,13 @@ def run_gpu(w: inputs.Workload, T: Optional[int] = None, layer: int = 0, pool=No
     logits = torch.from_numpy(li.logits).cuda()
     st = torch.from_numpy(np.asarray(slot_table, dtype=np.int32)).cuda()
     lay = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode)
+    from moe_expert_layer_renorm_b200 import _lib
+    _lib.device_status(clear=True)
     y = lay.forward(x, logits, st, pool)
     torch.cuda.synchronize()
+    detail = _lib.device_status_detail()
+    status = _lib.device_status(clear=True)
+    assert status == expect_status, f"device status {status} (detail {detail})"
     return GpuRun(lay, li.x_bits, li.logits, np.asarray(slot_table), pool, bf16_to_f64(y))
 
 

@@ -154,8 +154,7 @@ def test_non_resident_expert_sets_status(cuda_device):
     ids, _ = G.M.route(li.logits, w.k)
     st = st.copy()
     st[int(ids[0, 0])] = -1
-    G.run_gpu(w, pool=pool, slot_table=st, li=li)
-    assert _lib.device_status(clear=True) == _lib.FT_DEV_NOT_RESIDENT
+    G.run_gpu(w, pool=pool, slot_table=st, li=li, expect_status=_lib.FT_DEV_NOT_RESIDENT)
     # the library stays usable afterwards
     run = G.run_gpu(w)
     G.check_output(run, w.k)
