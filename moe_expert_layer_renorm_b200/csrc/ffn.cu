@@ -504,233 +504,4 @@ __global__ void __launch_bounds__(1024) ffn_schedule_kernel(
   for (int i = threadIdx.x; i < ncnt2; i += blockDim.x) counters2[i] = 0;
 }
 
-// --------------------------------------------------------------- host ---
-
-struct GemmShape { int bn, splits, sps, ws, bs, as, db; };
-
-struct FfnPlan {
-  bool decode;
-  GemmShape g1, g2;
-  int mt1, mt2, nkw1, nkw2, nkc1, nkc2;
-  long long max_tiles1, max_tiles2;
-  // workspace layout (byte offsets)
-  size_t off_h, off_units1, off_units2, off_counts, off_cnt1, off_cnt2, off_part1, off_part2, total;
-  long long max_units1, max_units2;
-};
-
-static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-static int choose_splits(double units_est, int nkw, int num_sms, int* sps_out) {
-  int s = 1;
-  if (units_est < num_sms) s = (int)ceil(num_sms / units_est);
-  s = std::max(1, std::min(s, nkw));
-  const int sps = (nkw + s - 1) / s;
-  *sps_out = sps;
-  return (nkw + sps - 1) / sps;
-}
-
-static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
-  FfnPlan pl{};
-  const long long P = (long long)T * k;
-  const double distinct = E * (1.0 - pow(1.0 - double(k) / E, double(T)));
-  const double mean_rows = distinct > 0 ? double(P) / distinct : 0.0;
-  pl.decode = mean_rows <= 32.0;
-  pl.mt1 = (I + 127) / 128;
-  pl.mt2 = (H + 127) / 128;
-  pl.nkw1 = (H + kKW - 1) / kKW;
-  pl.nkw2 = (I + kKW - 1) / kKW;
-  pl.nkc1 = H / kKC;
-  pl.nkc2 = I / kKC;
-  if (pl.decode) {
-    pl.g1 = {32, 1, 0, 5, 8, 4, 2};
-    pl.g2 = {32, 1, 0, 8, 8, 4, 2};
-  } else {
-    pl.g1 = {128, 1, 0, 3, 4, 4, 1};
-    pl.g2 = {128, 1, 0, 3, 6, 4, 2};
-  }
-  const double est_tiles1 = std::max(1.0, ceil(distinct) + (pl.decode ? 0.0 : double(P) / pl.g1.bn));
-  const double est_tiles2 = std::max(1.0, ceil(distinct) + (pl.decode ? 0.0 : double(P) / pl.g2.bn));
-  pl.g1.splits = choose_splits(est_tiles1 * pl.mt1, pl.nkw1, num_sms, &pl.g1.sps);
-  pl.g2.splits = choose_splits(est_tiles2 * pl.mt2, pl.nkw2, num_sms, &pl.g2.sps);
-  const long long active = std::min<long long>(E, P);
-  pl.max_tiles1 = active + P / pl.g1.bn;
-  pl.max_tiles2 = active + P / pl.g2.bn;
-  pl.max_units1 = pl.max_tiles1 * pl.mt1 * pl.g1.splits;
-  pl.max_units2 = pl.max_tiles2 * pl.mt2 * pl.g2.splits;
-  size_t o = 0;
-  pl.off_h = o;       o = align256(o + size_t(P) * I * 2);
-  pl.off_units1 = o;  o = align256(o + size_t(pl.max_units1) * 16);
-  pl.off_units2 = o;  o = align256(o + size_t(pl.max_units2) * 16);
-  pl.off_counts = o;  o = align256(o + 16);
-  pl.off_cnt1 = o;    o = align256(o + size_t(pl.max_tiles1 * pl.mt1) * 4 * 4);
-  pl.off_cnt2 = o;    o = align256(o + size_t(pl.max_tiles2 * pl.mt2) * 4 * 4);
-  pl.off_part1 = o;
-  if (pl.g1.splits > 1) o = align256(o + size_t(pl.max_units1) * 2 * 128 * pl.g1.bn * 4);
-  pl.off_part2 = o;
-  if (pl.g2.splits > 1) o = align256(o + size_t(pl.max_units2) * 1 * 128 * pl.g2.bn * 4);
-  pl.total = o;
-  return pl;
-}
-
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// codes: [rows, K/2] bytes per slot, 128 x 128-byte boxes, 128-byte swizzle.
-// scales: [rows, ld_scale] bytes per slot, 128 x 16-byte boxes.
-static bool make_weight_maps(const uint8_t* pool, const ft_nvfp4_slot_layout& L, int mat, int rows, int K,
-                             CUtensorMap* codes, CUtensorMap* scales) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint32_t elem_strides[3] = {1, 1, 1};
-  {
-    const cuuint64_t dims[3] = {cuuint64_t(K / 2), cuuint64_t(rows), cuuint64_t(L.num_slots)};
-    const cuuint64_t strides[2] = {cuuint64_t(K / 2), cuuint64_t(L.slot_bytes)};
-    const cuuint32_t box[3] = {128, 128, 1};
-    if (enc(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)(pool + L.codes_off[mat]), dims, strides, box,
-            elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
-  }
-  {
-    const cuuint64_t dims[3] = {cuuint64_t(L.ld_scale[mat]), cuuint64_t(rows), cuuint64_t(L.num_slots)};
-    const cuuint64_t strides[2] = {cuuint64_t(L.ld_scale[mat]), cuuint64_t(L.slot_bytes)};
-    const cuuint32_t box[3] = {16, 128, 1};
-    if (enc(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)(pool + L.scales_off[mat]), dims, strides, box,
-            elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
-  }
-  return true;
-}
-
-// Activation rows (bf16 [rows, K]) as the MMA's B operand, 64-column (128-byte)
-// boxes with the 128-byte swizzle: one-row boxes for tile::gather4, or
-// 16-row boxes for contiguous rows.
-static bool make_act_map(const void* base, int rows, int K, int box_rows, CUtensorMap* m) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
-  const cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
-  const cuuint32_t elem_strides[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <int NMAT, int BN, int WS, int BS, int AS, int DB>
-static cudaError_t launch_gemm(const FfnParams& p, int grid, const CUtensorMap& c0, const CUtensorMap& s0,
-                               const CUtensorMap& c1, const CUtensorMap& s1, const CUtensorMap& act,
-                               cudaStream_t s) {
-  ProfileScope prof(NMAT == 2 ? FT_KERNEL_GEMM_GATE_UP : FT_KERNEL_GEMM_DOWN, s);
-  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB>;
-  auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  kern<<<grid, kThreads, Cfg::kSmemBytes, s>>>(p, c0, s0, c1, s1, act);
-  return cudaGetLastError();
-}
-
-static int device_sm_count() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n;
-}
-
-static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, const int32_t* perm_src,
-                              const int32_t* offsets, const int32_t* slot_table, const void* pool_v,
-                              const ft_nvfp4_slot_layout& L, void* out_perm, void* ws, cudaStream_t s,
-                              const char** why) {
-  const int num_sms = device_sm_count();
-  const FfnPlan pl = plan_ffn(T, H, I, E, k, num_sms);
-  const uint8_t* pool = static_cast<const uint8_t*>(pool_v);
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  CUtensorMap tmc[3], tms[3];
-  const int rows[3] = {I, I, H}, Ks[3] = {H, H, I};
-  for (int m = 0; m < 3; ++m)
-    if (!make_weight_maps(pool, L, m, rows[m], Ks[m], &tmc[m], &tms[m])) {
-      *why = "cuTensorMapEncodeTiled failed for the slot pool";
-      return cudaErrorInvalidValue;
-    }
-  int4* units1 = reinterpret_cast<int4*>(w + pl.off_units1);
-  int4* units2 = reinterpret_cast<int4*>(w + pl.off_units2);
-  int* counts = reinterpret_cast<int*>(w + pl.off_counts);
-  int* cnt1 = reinterpret_cast<int*>(w + pl.off_cnt1);
-  int* cnt2 = reinterpret_cast<int*>(w + pl.off_cnt2);
-  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(w + pl.off_h);
-  {
-  ProfileScope prof(FT_KERNEL_SCHEDULE, s);
-  ffn_schedule_kernel<<<1, 1024, 0, s>>>(offsets, slot_table, E, L.num_slots, pl.g1.bn, pl.mt1, pl.g1.splits,
-                                         pl.g2.bn, pl.mt2, pl.g2.splits, units1, units2, counts, cnt1,
-                                         int(pl.max_tiles1 * pl.mt1 * 4), cnt2, int(pl.max_tiles2 * pl.mt2 * 4));
-  }
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-
-  CUtensorMap tm_x, tm_h;
-  if (!make_act_map(x, T, H, 1, &tm_x) || !make_act_map(h, T * k, I, 16, &tm_h)) {
-    *why = "cuTensorMapEncodeTiled failed for the activations";
-    return cudaErrorInvalidValue;
-  }
-  FfnParams p1{};
-  p1.perm_src = perm_src;
-  p1.k_top = k;
-  p1.K = H;
-  p1.M = I;
-  p1.nkw = pl.nkw1;
-  p1.nkc = pl.nkc1;
-  p1.splits = pl.g1.splits;
-  p1.stages_per_split = pl.g1.sps;
-  p1.units = units1;
-  p1.num_units = counts;
-  p1.slot_table = slot_table;
-  p1.pool = pool;
-  p1.slot_bytes = L.slot_bytes;
-  p1.global_off[0] = L.global_off[FT_GATE];
-  p1.global_off[1] = L.global_off[FT_UP];
-  p1.out = h;
-  p1.partials = reinterpret_cast<float*>(w + pl.off_part1);
-  p1.counters = cnt1;
-  const int grid1 = int(std::min<long long>(num_sms, pl.max_units1));
-
-  FfnParams p2 = p1;
-  p2.perm_src = nullptr;
-  p2.K = I;
-  p2.M = H;
-  p2.nkw = pl.nkw2;
-  p2.nkc = pl.nkc2;
-  p2.splits = pl.g2.splits;
-  p2.stages_per_split = pl.g2.sps;
-  p2.units = units2;
-  p2.num_units = counts + 1;
-  p2.global_off[0] = L.global_off[FT_DOWN];
-  p2.global_off[1] = L.global_off[FT_DOWN];
-  p2.out = out_perm;
-  p2.partials = reinterpret_cast<float*>(w + pl.off_part2);
-  p2.counters = cnt2;
-  const int grid2 = int(std::min<long long>(num_sms, pl.max_units2));
-
-  if (pl.decode) {
-    err = launch_gemm<2, 32, 5, 8, 4, 2>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
-    if (err == cudaSuccess) err = launch_gemm<1, 32, 8, 8, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
-  } else {
-    err = launch_gemm<2, 128, 3, 4, 4, 1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
-    if (err == cudaSuccess) err = launch_gemm<1, 128, 3, 6, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
-  }
-  return err;
-}
-
 }  // namespace ftmoe

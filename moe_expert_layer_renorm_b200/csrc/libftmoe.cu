@@ -12,5 +12,7 @@
 #include "combine.cu"
 #include "pack.cu"
 #include "ffn.cu"
+#include "decode.cu"
+#include "ffn_host.cu"
 #include "api.cu"
 #include "slots.cpp"
