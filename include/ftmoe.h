@@ -68,6 +68,7 @@ enum {
   FT_DEV_WAIT_TIMEOUT = 1,  /* an internal pipeline wait exceeded ~1 s */
   FT_DEV_NOT_RESIDENT = 2,  /* a non-empty expert group had slot -1 */
   FT_DEV_BAD_INDEX = 3,     /* an expert id or slot outside its range */
+  FT_DEV_F16_RANGE = 4,     /* an intermediate exceeded the f16 range (saturated) */
 };
 
 enum {
@@ -139,10 +140,14 @@ FT_API size_t ft_moe_permute_workspace_size(int T, int k, int E);
  * slot_pool + slot_table[e] * layout->slot_bytes:
  *   h[r]        = silu(gG * (Qg x_t)) * (gU * (Qu x_t))        (I values)
  *   out_perm[r] = gD * (Qd h[r])                                (H values, fp32)
- * where Q* are the E2M1*E4M3 dequantised weights (exact in bf16), g* the
- * fp32 global scales, products accumulate in fp32 on the tensor cores, and
- * h is rounded to bf16 before the down projection (it is that MMA's
- * operand).  The expert outputs stay fp32 so that the layer output meets
+ * where Q* are the E2M1*E4M3 dequantised weights, g* the fp32 global scales,
+ * and products accumulate in fp32 on the tensor cores.  The MMA operands are
+ * f16: every E2M1*E4M3 product is exact in f16; each token row of x is
+ * converted once, after a power-of-two prescale that puts its largest
+ * magnitude below 2^15 (exact for every element within 2^32 of that
+ * maximum, else an absolute error below 2^-41 of it); h is rounded to f16
+ * (values beyond the f16 range saturate and set FT_DEV_F16_RANGE).  The
+ * expert outputs stay fp32 so that the layer output meets
  * |y - y_exact| <= 1e-2 rms(y) + 1e-3: a bf16 rounding of them (or of y) alone
  * would already reach that bound at the tails of the output distribution.
  *   x              device bf16 [T, H]
@@ -264,7 +269,8 @@ enum {
   FT_KERNEL_GEMM_DOWN = 4,    /* grouped down GEMM */
   FT_KERNEL_COMBINE = 5,
   FT_KERNEL_PACK = 6,
-  FT_KERNEL_KINDS = 7,
+  FT_KERNEL_PREP = 7,         /* activations to f16 (inside ft_moe_ffn_nvfp4) */
+  FT_KERNEL_KINDS = 8,
 };
 
 typedef struct {

@@ -24,6 +24,7 @@ FT_DEV_OK = 0
 FT_DEV_WAIT_TIMEOUT = 1
 FT_DEV_NOT_RESIDENT = 2
 FT_DEV_BAD_INDEX = 3
+FT_DEV_F16_RANGE = 4
 
 FT_ROUTE_SOFTMAX_RENORM = 0
 FT_ROUTE_TOPK_SOFTMAX = 1
@@ -51,11 +52,11 @@ class SlotLayout(ctypes.Structure):
     ]
 
 
-FT_KERNEL_NAMES = ("route", "permute", "schedule", "gemm_gate_up", "gemm_down", "combine", "pack")
+FT_KERNEL_NAMES = ("route", "permute", "schedule", "gemm_gate_up", "gemm_down", "combine", "pack", "prep_x")
 
 
 class Profile(ctypes.Structure):
-    _fields_ = [("launches", c_int64 * 7), ("timed", c_int64 * 7), ("total_ms", ctypes.c_double * 7)]
+    _fields_ = [("launches", c_int64 * 8), ("timed", c_int64 * 8), ("total_ms", ctypes.c_double * 8)]
 
 
 class SlotStats(ctypes.Structure):

@@ -8,16 +8,18 @@
 // tile must be written to and read back from shared memory, which saturates
 // its bandwidth first.  Streaming at HBM rate needs ~35 weights per clock per
 // SM, so the weights instead flow from TMA-staged shared memory through
-// registers straight into warp-level MMA fragments (mma.sync m16n8k16, bf16 x
-// bf16 -> fp32): 256 weights per instruction, no shared-memory round trip for
+// registers straight into warp-level MMA fragments (mma.sync m16n8k16, f16 x
+// f16 -> fp32): 256 weights per instruction, no shared-memory round trip for
 // the dequantised values, and the tensor cores do the FMAs.
 //
 // CTA tile: 256 weight rows (16 compute warps x 16 rows) x all of the unit's K,
-// for one expert's group of <= 16 token rows (two n = 8 MMA tiles).
-//   warp 0     TMA: codes (2 x 128 rows x 128 B, 128-byte swizzle) and scales
-//              (2 x 128 rows x 16 B) of each matrix, 256 K per stage
-//   warp 1     TMA: the group's token rows for the same 256 K (gather4 of x
-//              rows for the gate/up GEMM, 16-row tiles of h for the down GEMM)
+// for one expert's group of <= 16 token rows (two n = 8 MMA tiles).  A stage
+// holds one matrix's 256 rows for 256 K plus the token rows for that K, so
+// the gate/up GEMM alternates gate and up stages.
+//   warp 0     TMA: codes (256 rows x 128 B, 128-byte swizzle) and scales
+//              (256 rows x 16 B) of one matrix, 256 K per stage
+//   warp 1     TMA: the group's 16 token rows for the same 256 K (16-row tiles
+//              of the permuted f16 activations, or of h)
 //   warps 2-17 compute: warp w owns rows 16w .. 16w + 15 of the tile
 //
 // K permutation.  A dot product may visit K in any order as long as both
@@ -28,7 +30,7 @@
 // two scale bytes), and its token values are 32 consecutive K of the token row
 // (four 16-byte loads).
 #include <cuda.h>
-#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include "sm100.cuh"
 
 namespace ftmoe {
@@ -40,9 +42,9 @@ constexpr int kDecStageK = 256;
 
 template <int NMAT, int STAGES>
 struct DecCfg {
-  static constexpr int kWBoxBytes = kMatStageBytes;                  // one 128-row box: codes + scales
-  static constexpr int kWStageBytes = NMAT * 2 * kWBoxBytes;         // 2 boxes per matrix
-  static constexpr int kBBoxBytes = kDecBN * 128;                    // 64 K x 16 rows of bf16
+  static constexpr int kCodes = kDecRows * 128;                      // 256 rows x 128 B of codes
+  static constexpr int kWStageBytes = kCodes + kDecRows * 16;        // + 256 rows x 16 B of scales
+  static constexpr int kBBoxBytes = kDecBN * 128;                    // 64 K x 16 rows of f16
   static constexpr int kBStageBytes = 4 * kBBoxBytes;                // 256 K
   static constexpr int kStageBytes = kWStageBytes + kBStageBytes;    // multiple of 1024
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + 2 * STAGES * 8 + 64;
@@ -50,10 +52,10 @@ struct DecCfg {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -70,7 +72,6 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::kStageBytes);
   uint64_t* empty = full + STAGES;
   int* abort_flag = reinterpret_cast<int*>(empty + STAGES);
-  __shared__ int rowidx[kDecBN];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -106,21 +107,15 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
         int e, mt, rb, nr, ws0, ws1;
         unit_range(u, e, mt, rb, nr, ws0, ws1);
         const int slot = __ldg(p.slot_table + e);
-        for (int ws = ws0; ws < ws1; ++ws, ++si) {
-          const int s = si % STAGES;
-          if (!(ok = ab.wait(&empty[s], ((si / STAGES) & 1) ^ 1, kTagWEmpty, si, u))) break;
-          mbar_arrive_expect_tx(&full[s], Cfg::kWStageBytes);
-          uint8_t* st = smem + s * Cfg::kStageBytes;
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-            for (int bx = 0; bx < 2; ++bx) {
-              uint8_t* dst = st + (m * 2 + bx) * Cfg::kWBoxBytes;
-              const int y = mt * kDecRows + bx * 128;
-              tma_load_3d(dst, tmc[m], &full[s], ws * 128, y, slot);
-              tma_load_3d(dst + kCodesBytes, tms[m], &full[s], ws * 16, y, slot);
-            }
-        }
+        for (int ws = ws0; ws < ws1 && ok; ++ws)
+          for (int m = 0; m < NMAT; ++m, ++si) {
+            const int s = si % STAGES;
+            if (!(ok = ab.wait(&empty[s], ((si / STAGES) & 1) ^ 1, kTagWEmpty, si, u))) break;
+            mbar_arrive_expect_tx(&full[s], Cfg::kWStageBytes);
+            uint8_t* st = smem + s * Cfg::kStageBytes;
+            tma_load_3d(st, tmc[m], &full[s], ws * 128, mt * kDecRows, slot);
+            tma_load_3d(st + Cfg::kCodes, tms[m], &full[s], ws * 16, mt * kDecRows, slot);
+          }
       }
       for (uint32_t j = (si > STAGES ? si - STAGES : 0); j < si; ++j) {   // drain
         const uint64_t t0 = globaltimer_ns();
@@ -129,42 +124,23 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
     }
   } else if (warp == 1) {
     // ------------------------------------------------- token TMA ---
-    uint32_t si = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      int e, mt, rb, nr, ws0, ws1;
-      unit_range(u, e, mt, rb, nr, ws0, ws1);
-      if (lane < kDecBN) {
-        const int r = rb + min(lane, nr - 1);
-        rowidx[lane] = p.perm_src ? __ldg(p.perm_src + r) / p.k_top : r;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        for (int ws = ws0; ws < ws1; ++ws, ++si) {
+    if (lane == 0) {
+      uint32_t si = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        int e, mt, rb, nr, ws0, ws1;
+        unit_range(u, e, mt, rb, nr, ws0, ws1);
+        for (int q = ws0 * NMAT; q < ws1 * NMAT; ++q, ++si) {
+          const int ws = q / NMAT;
           const int s = si % STAGES;
           if (!(ok = ab.wait(&empty[s], ((si / STAGES) & 1) ^ 1, kTagBEmpty, si, u))) break;
           mbar_arrive_expect_tx(&full[s], Cfg::kBStageBytes);
           uint8_t* bst = smem + s * Cfg::kStageBytes + Cfg::kWStageBytes;
 #pragma unroll
-          for (int bx = 0; bx < 4; ++bx) {
-            uint8_t* dst = bst + bx * Cfg::kBBoxBytes;
-            const int k = ws * kDecStageK + bx * 64;
-            if (p.perm_src) {
-#pragma unroll
-              for (int n = 0; n < kDecBN; n += 4)
-                tma_gather4(dst + n * 128, &tm_act, &full[s], k, rowidx[n], rowidx[n + 1], rowidx[n + 2],
-                            rowidx[n + 3]);
-            } else {
-              tma_load_2d(dst, &tm_act, &full[s], k, rb);
-            }
-          }
+          for (int bx = 0; bx < 4; ++bx)
+            tma_load_2d(bst + bx * Cfg::kBBoxBytes, &tm_act, &full[s], ws * kDecStageK + bx * 64, rb);
         }
       }
-      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-      si = __shfl_sync(0xFFFFFFFFu, si, 0);
-      __syncwarp();
-    }
-    if (lane == 0) {
       for (uint32_t j = (si > STAGES ? si - STAGES : 0); j < si; ++j) {
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1) && globaltimer_ns() - t0 < 1000000000ull) {}
@@ -174,8 +150,7 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
     // --------------------------------------------------- compute ---
     const int cw = warp - 2;                 // 0..15
     const int g = lane >> 2, t = lane & 3;   // mma quad layout
-    const int bx = cw >> 3;                  // which 128-row box
-    const int r_lo = 16 * (cw & 7) + g;      // rows within the box
+    const int r_lo = 16 * cw + g;            // rows of the 256-row tile
     const int r_hi = r_lo + 8;
     uint32_t si = 0;
     bool ok = true;
@@ -191,56 +166,55 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.0f;
 
-      for (int ws = ws0; ws < ws1; ++ws, ++si) {
+      for (int q = ws0 * NMAT; q < ws1 * NMAT; ++q, ++si) {
+        const int m = q % NMAT;
         const int s = si % STAGES;
-        if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&full[s], (si / STAGES) & 1, kTagWFull, si, u)))) break;
+          if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&full[s], (si / STAGES) & 1, kTagWFull, si, u)))) break;
         const uint8_t* st = smem + s * Cfg::kStageBytes;
         const uint8_t* bst = st + Cfg::kWStageBytes;
+        // one matrix's 256 rows x 256 K against the unit's token rows
+        auto stage_mma = [&](float (&am)[2][4]) {
+          const int n0 = g, n1 = 8 + g;   // token rows of MMA tiles 0 and 1
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          // token fragments: 32 consecutive K of token rows g (tile 0) and 8 + g (tile 1)
-          uint32_t bf[2][16];
-          const uint8_t* bbox = bst + (2 * h + (t >> 1)) * Cfg::kBBoxBytes;
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            const int n = 8 * nt + g;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint4 v = *reinterpret_cast<const uint4*>(bbox + n * 128 + ((((t & 1) * 4 + c) ^ (n & 7)) << 4));
-              bf[nt][4 * c] = v.x; bf[nt][4 * c + 1] = v.y; bf[nt][4 * c + 2] = v.z; bf[nt][4 * c + 3] = v.w;
-            }
-          }
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            const uint8_t* wb = st + (m * 2 + bx) * Cfg::kWBoxBytes;
+          for (int h = 0; h < 2; ++h) {
+            const uint8_t* bbox = bst + (2 * h + (t >> 1)) * Cfg::kBBoxBytes;
             const int chunk = 4 * h + t;   // 16-byte chunk of the 128-byte row: 32 codes
-            const uint4 clo = *reinterpret_cast<const uint4*>(wb + r_lo * 128 + ((chunk ^ (r_lo & 7)) << 4));
-            const uint4 chi = *reinterpret_cast<const uint4*>(wb + r_hi * 128 + ((chunk ^ (r_hi & 7)) << 4));
-            const uint32_t slo = *reinterpret_cast<const uint16_t*>(wb + kCodesBytes + r_lo * 16 + 8 * h + 2 * t);
-            const uint32_t shi = *reinterpret_cast<const uint16_t*>(wb + kCodesBytes + r_hi * 16 + 8 * h + 2 * t);
-            const uint32_t s_lo[2] = {e4m3_pair_to_f16x2(slo & 0xFFu), e4m3_pair_to_f16x2(slo >> 8)};
-            const uint32_t s_hi[2] = {e4m3_pair_to_f16x2(shi & 0xFFu), e4m3_pair_to_f16x2(shi >> 8)};
+            const uint4 clo = *reinterpret_cast<const uint4*>(st + r_lo * 128 + ((chunk ^ (r_lo & 7)) << 4));
+            const uint4 chi = *reinterpret_cast<const uint4*>(st + r_hi * 128 + ((chunk ^ (r_hi & 7)) << 4));
+            const uint8_t* sc = st + Cfg::kCodes;
+            const uint32_t slo = *reinterpret_cast<const uint16_t*>(sc + r_lo * 16 + 8 * h + 2 * t);
+            const uint32_t shi = *reinterpret_cast<const uint16_t*>(sc + r_hi * 16 + 8 * h + 2 * t);
             const uint32_t wlo[4] = {clo.x, clo.y, clo.z, clo.w};
             const uint32_t whi[4] = {chi.x, chi.y, chi.z, chi.w};
 #pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {      // word wd holds the codes of MMAs 2 wd and 2 wd + 1
+            for (int wd = 0; wd < 4; ++wd) {   // word wd: codes of MMAs 2 wd and 2 wd + 1
+              // token values for those two MMAs: 16-byte chunk wd of the thread's 64 bytes
+              const int cb = (t & 1) * 4 + wd;
+              const uint4 b0 = *reinterpret_cast<const uint4*>(bbox + n0 * 128 + ((cb ^ (n0 & 7)) << 4));
+              uint4 b1 = make_uint4(0u, 0u, 0u, 0u);
+              if (ntiles > 1) b1 = *reinterpret_cast<const uint4*>(bbox + n1 * 128 + ((cb ^ (n1 & 7)) << 4));
+              const uint32_t sl = e4m3_pair_to_f16x2(wd < 2 ? (slo & 0xFFu) : (slo >> 8));
+              const uint32_t sh = e4m3_pair_to_f16x2(wd < 2 ? (shi & 0xFFu) : (shi >> 8));
               uint32_t qlo[4], qhi[4];
               e2m1x8_to_f16x2(wlo[wd], qlo);
               e2m1x8_to_f16x2(whi[wd], qhi);
-              const int sb = wd >> 1;             // MMAs 0..3 use the first scale block, 4..7 the second
-#pragma unroll
-              for (int half = 0; half < 2; ++half) {
-                const int i = 2 * wd + half;
-                const uint32_t a0 = f16x2_to_bf16x2(hmul2_f16(qlo[2 * half], s_lo[sb]));
-                const uint32_t a1 = f16x2_to_bf16x2(hmul2_f16(qhi[2 * half], s_hi[sb]));
-                const uint32_t a2 = f16x2_to_bf16x2(hmul2_f16(qlo[2 * half + 1], s_lo[sb]));
-                const uint32_t a3 = f16x2_to_bf16x2(hmul2_f16(qhi[2 * half + 1], s_hi[sb]));
-                mma_bf16_16816(acc[m][0], a0, a1, a2, a3, bf[0][2 * i], bf[0][2 * i + 1]);
-                if (ntiles > 1) mma_bf16_16816(acc[m][1], a0, a1, a2, a3, bf[1][2 * i], bf[1][2 * i + 1]);
+              {
+                const uint32_t a0 = hmul2_f16(qlo[0], sl), a1 = hmul2_f16(qhi[0], sh);
+                const uint32_t a2 = hmul2_f16(qlo[1], sl), a3 = hmul2_f16(qhi[1], sh);
+                mma_f16_16816(am[0], a0, a1, a2, a3, b0.x, b0.y);
+                if (ntiles > 1) mma_f16_16816(am[1], a0, a1, a2, a3, b1.x, b1.y);
+              }
+              {
+                const uint32_t a0 = hmul2_f16(qlo[2], sl), a1 = hmul2_f16(qhi[2], sh);
+                const uint32_t a2 = hmul2_f16(qlo[3], sl), a3 = hmul2_f16(qhi[3], sh);
+                mma_f16_16816(am[0], a0, a1, a2, a3, b0.z, b0.w);
+                if (ntiles > 1) mma_f16_16816(am[1], a0, a1, a2, a3, b1.z, b1.w);
               }
             }
           }
-        }
+        };
+        if (NMAT == 1 || m == 0) stage_mma(acc[0]);
+        else stage_mma(acc[NMAT - 1]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
@@ -252,7 +226,7 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
       float gsc[NMAT];
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) gsc[m] = __ldg(reinterpret_cast<const float*>(sbase + p.global_off[m]));
-      const int f0 = mt * kDecRows + 128 * bx + r_lo;   // features of c0/c1 (f0) and c2/c3 (f0 + 8)
+      const int f0 = mt * kDecRows + r_lo;   // features of c0/c1 (f0) and c2/c3 (f0 + 8)
       if (p.splits > 1) {
         // partials[u][m][n][256 rows]
 #pragma unroll
@@ -262,7 +236,7 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int n = 8 * nt + 2 * t + (i & 1);
-              const int rr = 128 * bx + r_lo + (i >> 1) * 8;
+              const int rr = r_lo + (i >> 1) * 8;
               if (n < nr) p.partials[((size_t(u) * NMAT + m) * kDecBN + n) * kDecRows + rr] = acc[m][nt][i];
             }
         __threadfence();
@@ -280,7 +254,7 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int n = 8 * nt + 2 * t + (i & 1);
-              const int rr = 128 * bx + r_lo + (i >> 1) * 8;
+              const int rr = r_lo + (i >> 1) * 8;
               float a = 0.0f;
               if (n < nr)
                 for (int sp = 0; sp < p.splits; ++sp)
@@ -297,8 +271,12 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
           const int f = f0 + (i >> 1) * 8;
           if (n < nr && f < p.M) {
             float r;
-            if (NMAT == 2) r = silu_mul(gsc[0] * acc[0][nt][i], gsc[NMAT - 1] * acc[NMAT - 1][nt][i]);
-            else r = gsc[0] * acc[0][nt][i];
+            if (NMAT == 2) {
+              const float ts = token_factor(p, rb + n);
+              r = silu_mul(gsc[0] * ts * acc[0][nt][i], gsc[NMAT - 1] * ts * acc[NMAT - 1][nt][i]);
+            } else {
+              r = gsc[0] * acc[0][nt][i];
+            }
             store_out<NMAT>(p.out, size_t(rb + n) * p.M + f, r);
           }
         }

@@ -8,10 +8,10 @@
 // Data path of one CTA (persistent; 16 warps):
 //   warp 0      TMA: packed E2M1 codes (128 rows x 128 B, 128-byte swizzle)
 //               and E4M3 scales (128 rows x 16 B) of each matrix, 256 K per stage
-//   warp 2      TMA: the unit's token rows (bf16, 64 K per chunk) into
-//               128-byte-swizzled K-major shared memory (the MMA's B operand);
-//               GEMM1 gathers x rows through perm_src four at a time
-//               (tile::gather4), GEMM2 loads 16-row tiles of h
+//   warp 2      TMA: the unit's token rows (f16, 64 K per chunk) into
+//               128-byte-swizzled K-major shared memory (the MMA's B operand),
+//               16-row tiles of the permuted f16 activations (GEMM1) or of h
+//               (GEMM2); both are stored in permuted row order
 //   warps 4-11  dequantise one 64-K chunk per step: E2M1 -> f16 (cvt) times the
 //               E4M3 block scale (exact in f16), widened to bf16 (exact), and
 //               stored with tcgen05.st straight into tensor memory, where the
@@ -43,6 +43,8 @@ constexpr int kMatStageBytes = kCodesBytes + kScaleBytes;   // 18 KB, multiple o
 constexpr int kThreads = 512;
 
 struct FfnParams {
+  const float* tokscale;      // GEMM1: per-token factor undoing the f16 prescale of x
+  const int* any_scaled;      // GEMM1: nonzero when some token was prescaled
   const int32_t* perm_src;    // GEMM1: row -> pair (token = pair / k_top); GEMM2: null (row -> row)
   int k_top;
   int K;                      // reduction length
@@ -57,7 +59,7 @@ struct FfnParams {
   const uint8_t* pool;
   long long slot_bytes;
   long long global_off[2];
-  void* out;                  // GEMM1: h bf16 [P, M]; GEMM2: out_perm fp32 [P, M]
+  void* out;                  // GEMM1: h f16 [P, M]; GEMM2: out_perm fp32 [P, M]
   float* partials;            // split-K partial accumulators
   int* counters;              // split-K arrival counters, 4 per (tile, m_tile): one per epilogue warp
 };
@@ -106,7 +108,9 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
 }
 
 // 64 codes (two 16-byte words of one row) and their 4 scale bytes -> 32
-// bf16x2 words, word c holding k = 2c (low half) and 2c + 1 (high half).
+// f16x2 words, word c holding k = 2c (low half) and 2c + 1 (high half).
+// Every E2M1 x E4M3 product (at most 6 significant bits, magnitude in
+// [2^-10, 2688]) is an exact f16, so the products carry no rounding.
 __device__ __forceinline__ void dequant_chunk(const uint4& c0, const uint4& c1, uint32_t sc,
                                               uint32_t (&o)[32]) {
   const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -118,7 +122,7 @@ __device__ __forceinline__ void dequant_chunk(const uint4& c0, const uint4& c1, 
       uint32_t q[4];
       e2m1x8_to_f16x2(w[2 * b + h], q);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) o[(2 * b + h) * 4 + j] = f16x2_to_bf16x2(hmul2_f16(q[j], s2));
+      for (int j = 0; j < 4; ++j) o[(2 * b + h) * 4 + j] = hmul2_f16(q[j], s2);
     }
   }
 }
@@ -152,12 +156,27 @@ struct Abort {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
-// GEMM1 stores h in bf16 (it is the next MMA's operand); GEMM2 stores the
-// expert outputs in fp32 so that only the combine's own fp32 sum rounds them.
+// GEMM1 stores h in f16 (it is the next MMA's operand; a value beyond the f16
+// range saturates and records FT_DEV_F16_RANGE); GEMM2 stores the expert
+// outputs in fp32 so that only the combine's own fp32 sum rounds them.
 template <int NMAT>
 __device__ __forceinline__ void store_out(void* out, size_t idx, float v) {
-  if (NMAT == 2) static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
-  else static_cast<float*>(out)[idx] = v;
+  if (NMAT == 2) {
+    if (fabsf(v) > 65504.0f) {
+      set_device_status(FT_DEV_F16_RANGE);
+      v = copysignf(65504.0f, v);
+    }
+    static_cast<__half*>(out)[idx] = __float2half_rn(v);
+  } else {
+    static_cast<float*>(out)[idx] = v;
+  }
+}
+
+// Factor undoing the power-of-two prescale of token row `row` of a group
+// (GEMM1 only; 1 when no token needed a prescale).
+__device__ __forceinline__ float token_factor(const FfnParams& p, int row) {
+  if (p.perm_src == nullptr || *p.any_scaled == 0) return 1.0f;
+  return __ldg(p.tokscale + __ldg(p.perm_src + row) / p.k_top);
 }
 
 template <int NMAT, int BN, int WS, int BS, int AS, int DB>
@@ -170,8 +189,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* w_smem = smem;
   uint8_t* b_smem = smem + Cfg::kWBytes;
-  int* rowidx = reinterpret_cast<int*>(b_smem + Cfg::kBBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(rowidx + BN);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + Cfg::kBBytes);
   uint64_t* w_full = bars;
   uint64_t* w_empty = w_full + WS;
   uint64_t* b_full = w_empty + WS;
@@ -259,7 +277,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
         if (!(ok = ab.wait(&d_empty[ds], ((di / DB) & 1) ^ 1, kTagDEmpty, di, u))) break;
         tc_fence_after();
         const int n_eff = (nr + 15) & ~15;
-        const uint32_t idesc = make_idesc_f16(128, n_eff);
+        const uint32_t idesc = make_idesc_f16(128, n_eff, /*f16 operands=*/true);
         for (int c = kc0; c < kc1; ++c, ++q) {
           const int as = q % AS, bs = q % BS;
           if (!(ok = ab.wait(&a_full[as], (q / AS) & 1, kTagAFull, q, u))) break;
@@ -291,43 +309,26 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
     }
   } else if (warp == 2) {
     // --------------------------------------------- B (token) producer ---
-    // The lanes look up the unit's token rows; lane 0 issues one TMA per
-    // 4 rows (GEMM1, gathered x rows) or per 16 rows (GEMM2, contiguous h
-    // rows) for every 64-K chunk.  Rows past the group end but below the
-    // MMA's N repeat the last real row (their results are never stored).
+    // Lane 0 issues one 16-row TMA tile per 16 rows for every 64-K chunk.
+    // Rows past the group end but below the MMA's N are other groups' rows
+    // (or zero fill past the last row): finite, and their results are never
+    // stored.
     uint32_t q = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      int e, mt, rb, nr, ws0, ws1, kc0, kc1;
-      unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
-      const int n_eff = (nr + 15) & ~15;
-      for (int n = lane; n < n_eff; n += 32) {
-        const int r = rb + min(n, nr - 1);
-        rowidx[n] = p.perm_src ? __ldg(p.perm_src + r) / p.k_top : r;
-      }
-      __syncwarp();
-      if (lane == 0) {
+    if (lane == 0) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        int e, mt, rb, nr, ws0, ws1, kc0, kc1;
+        unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+        const int n_eff = (nr + 15) & ~15;
         for (int c = kc0; c < kc1; ++c, ++q) {
           const int bs = q % BS;
           if (!(ok = ab.wait(&b_empty[bs], ((q / BS) & 1) ^ 1, kTagBEmpty, q, u))) break;
           mbar_arrive_expect_tx(&b_full[bs], uint32_t(n_eff) * 128u);
           uint8_t* dst = b_smem + bs * Cfg::kBStageBytes;
-          const int k0 = c * kKC;
-          if (p.perm_src) {
-            for (int n = 0; n < n_eff; n += 4)
-              tma_gather4(dst + n * 128, &tm_act, &b_full[bs], k0, rowidx[n], rowidx[n + 1], rowidx[n + 2],
-                          rowidx[n + 3]);
-          } else {
-            for (int n = 0; n < n_eff; n += 16) tma_load_2d(dst + n * 128, &tm_act, &b_full[bs], k0, rb + n);
-          }
+          for (int n = 0; n < n_eff; n += 16) tma_load_2d(dst + n * 128, &tm_act, &b_full[bs], c * kKC, rb + n);
         }
       }
-      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-      q = __shfl_sync(0xFFFFFFFFu, q, 0);
-      __syncwarp();
-    }
-    if (lane == 0) {   // drain: the last copy into every B stage has landed
-      for (uint32_t j = (q > BS ? q - BS : 0); j < q; ++j) {
+      for (uint32_t j = (q > BS ? q - BS : 0); j < q; ++j) {   // drain
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&b_full[j % BS], (j / BS) & 1) && globaltimer_ns() - t0 < 1000000000ull) {}
       }
@@ -412,8 +413,12 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
               p.partials[(size_t(u) * NMAT + m) * 128 * BN + size_t(n) * 128 + row] = __uint_as_float(v[m][i]);
           } else if (feat < p.M) {
             float r;
-            if (NMAT == 2) r = silu_mul(gsc[0] * __uint_as_float(v[0][i]), gsc[NMAT - 1] * __uint_as_float(v[NMAT - 1][i]));
-            else r = gsc[0] * __uint_as_float(v[0][i]);
+            if (NMAT == 2) {
+              const float ts = token_factor(p, rb + n);
+              r = silu_mul(gsc[0] * ts * __uint_as_float(v[0][i]), gsc[NMAT - 1] * ts * __uint_as_float(v[NMAT - 1][i]));
+            } else {
+              r = gsc[0] * __uint_as_float(v[0][i]);
+            }
             store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
           }
         }
@@ -443,8 +448,12 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
             }
             if (feat < p.M) {
               float r;
-              if (NMAT == 2) r = silu_mul(gsc[0] * acc[0], gsc[NMAT - 1] * acc[NMAT - 1]);
-              else r = gsc[0] * acc[0];
+              if (NMAT == 2) {
+                const float ts = token_factor(p, rb + n);
+                r = silu_mul(gsc[0] * ts * acc[0], gsc[NMAT - 1] * ts * acc[NMAT - 1]);
+              } else {
+                r = gsc[0] * acc[0];
+              }
               store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
             }
           }
@@ -459,6 +468,62 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------ x to f16 ---
+
+// One warp per permuted row r (token t = perm_src[r] / k): writes
+// x_perm[r] = f16(x[t] * 2^-s_t) and tokscale[t] = 2^s_t, with s_t >= 0 the
+// smallest shift that brings max|x[t]| below 2^15.  The f16 conversion is
+// then exact for every element of the row within a factor 2^32 of the row's
+// largest magnitude (bf16 has 8 significant bits, f16 subnormals reach
+// 2^-24); smaller elements round with an absolute error below 2^-41 max|x[t]|.
+// Rows in permuted order make each expert group's tokens one contiguous
+// block, so the GEMM loads them as plain tiles.
+__global__ void __launch_bounds__(256) prep_x_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_src,
+                                                     int P, int k_top, int H, uint4* __restrict__ x_perm,
+                                                     float* __restrict__ tokscale, int* __restrict__ any_scaled) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (r >= P) return;
+  const int t = __ldg(perm_src + r) / k_top;
+  const int nv = H / 8;
+  const uint4* row = x + size_t(t) * nv;
+  float m = 0.0f;
+  for (int c = lane; c < nv; c += 32) {
+    const uint4 v = __ldg(row + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+  int shift = 0;
+  if (m >= 32768.0f && m <= 3.0e38f) {          // finite and too large for f16
+    int e;
+    frexpf(m, &e);                               // m = f * 2^e, f in [0.5, 1)
+    shift = e - 15;                              // m * 2^-shift < 2^15
+  } else if (!(m <= 3.0e38f)) {
+    set_device_status(FT_DEV_F16_RANGE);         // inf or nan input
+  }
+  const float f = ldexpf(1.0f, -shift);
+  if (lane == 0) {
+    tokscale[t] = ldexpf(1.0f, shift);           // every row of token t writes the same value
+    if (shift) atomicOr(any_scaled, 1);
+  }
+  uint4* out = x_perm + size_t(r) * nv;
+  for (int c = lane; c < nv; c += 32) {
+    const uint4 v = __ldg(row + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __half2 h = __floats2half2_rn(__uint_as_float(w[q] << 16) * f, __uint_as_float(w[q] & 0xFFFF0000u) * f);
+      o[q] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    out[c] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 

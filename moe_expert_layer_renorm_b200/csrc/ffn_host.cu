@@ -17,20 +17,33 @@ struct FfnPlan {
   int mt1, mt2, nkw1, nkw2, nkc1, nkc2;
   long long max_tiles1, max_tiles2;
   // workspace layout (byte offsets)
-  size_t off_h, off_units1, off_units2, off_counts, off_cnt1, off_cnt2, off_part1, off_part2, total;
+  size_t off_h, off_x16, off_tokscale, off_units1, off_units2, off_counts, off_cnt1, off_cnt2, off_part1, off_part2,
+      total;
   long long max_units1, max_units2;
   int cnt_per;
 };
 
 static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Split-K factor: a divisor of the K-stage count (all units of one launch do
+// equal work) that minimises the makespan of the persistent grid, i.e.
+// ceil(units * S / SMs) / (units * S / SMs), with a small charge per split
+// for the partial sums it writes and reduces.
 static int choose_splits(double units_est, int nkw, int num_sms, int* sps_out) {
-  int s = 1;
-  if (units_est < num_sms) s = (int)ceil(num_sms / units_est);
-  s = std::max(1, std::min(s, nkw));
-  const int sps = (nkw + s - 1) / s;
-  *sps_out = sps;
-  return (nkw + sps - 1) / sps;
+  int best = 1;
+  double best_cost = 1e30;
+  if (units_est >= 2.0 * num_sms) {   // enough parallelism: partial sums would only add traffic
+    *sps_out = nkw;
+    return 1;
+  }
+  for (int s = 1; s <= std::min(nkw, 16); ++s) {
+    if (nkw % s) continue;
+    const double work = units_est * s / num_sms;   // waves of equal units
+    const double cost = ceil(work - 1e-9) / work * (1.0 + 0.08 * (s - 1));
+    if (cost < best_cost - 1e-12) { best_cost = cost; best = s; }
+  }
+  *sps_out = nkw / best;
+  return best;
 }
 
 // Variant choice: groups of a few token rows (mean rows per active expert
@@ -53,7 +66,7 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   pl.nkc1 = H / kKC;
   pl.nkc2 = I / kKC;
   if (pl.decode) {
-    pl.g1 = {kDecBN, 1, 0, 2, 0, 0, 0};
+    pl.g1 = {kDecBN, 1, 0, 4, 0, 0, 0};
     pl.g2 = {kDecBN, 1, 0, 4, 0, 0, 0};
   } else {
     pl.g1 = {128, 1, 0, 3, 4, 4, 1};
@@ -76,9 +89,11 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   const size_t part_unit2 = pl.decode ? size_t(1) * kDecBN * kDecRows * 4 : size_t(1) * 128 * pl.g2.bn * 4;
   size_t o = 0;
   pl.off_h = o;       o = align256(o + size_t(P) * I * 2);
+  pl.off_x16 = o;     o = align256(o + size_t(P) * H * 2);   // f16 activations, permuted rows
+  pl.off_tokscale = o; o = align256(o + size_t(T) * 4);
   pl.off_units1 = o;  o = align256(o + size_t(pl.max_units1) * 16);
   pl.off_units2 = o;  o = align256(o + size_t(pl.max_units2) * 16);
-  pl.off_counts = o;  o = align256(o + 16);
+  pl.off_counts = o;  o = align256(o + 16);   // [0] units of GEMM1, [1] of GEMM2, [2] any token prescaled
   pl.off_cnt1 = o;    o = align256(o + size_t(pl.max_tiles1 * pl.mt1) * cnt_per * 4);
   pl.off_cnt2 = o;    o = align256(o + size_t(pl.max_tiles2 * pl.mt2) * cnt_per * 4);
   pl.off_part1 = o;
@@ -105,14 +120,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // codes: [rows, K/2] bytes per slot, 128 x 128-byte boxes, 128-byte swizzle.
 // scales: [rows, ld_scale] bytes per slot, 128 x 16-byte boxes.
 static bool make_weight_maps(const uint8_t* pool, const ft_nvfp4_slot_layout& L, int mat, int rows, int K,
-                             CUtensorMap* codes, CUtensorMap* scales) {
+                             int box_rows, CUtensorMap* codes, CUtensorMap* scales) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint32_t elem_strides[3] = {1, 1, 1};
   {
     const cuuint64_t dims[3] = {cuuint64_t(K / 2), cuuint64_t(rows), cuuint64_t(L.num_slots)};
     const cuuint64_t strides[2] = {cuuint64_t(K / 2), cuuint64_t(L.slot_bytes)};
-    const cuuint32_t box[3] = {128, 128, 1};
+    const cuuint32_t box[3] = {128, cuuint32_t(box_rows), 1};
     if (enc(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)(pool + L.codes_off[mat]), dims, strides, box,
             elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -121,7 +136,7 @@ static bool make_weight_maps(const uint8_t* pool, const ft_nvfp4_slot_layout& L,
   {
     const cuuint64_t dims[3] = {cuuint64_t(L.ld_scale[mat]), cuuint64_t(rows), cuuint64_t(L.num_slots)};
     const cuuint64_t strides[2] = {cuuint64_t(L.ld_scale[mat]), cuuint64_t(L.slot_bytes)};
-    const cuuint32_t box[3] = {16, 128, 1};
+    const cuuint32_t box[3] = {16, cuuint32_t(box_rows), 1};
     if (enc(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)(pool + L.scales_off[mat]), dims, strides, box,
             elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -133,14 +148,14 @@ static bool make_weight_maps(const uint8_t* pool, const ft_nvfp4_slot_layout& L,
 // Activation rows (bf16 [rows, K]) as the MMA's B operand, 64-column (128-byte)
 // boxes with the 128-byte swizzle: one-row boxes for tile::gather4, or
 // 16-row boxes for contiguous rows.
-static bool make_act_map(const void* base, int rows, int K, int box_rows, CUtensorMap* m) {
+static bool make_act_map(const void* base, int rows, int K, int box_rows, CUtensorMap* m) {  // f16 rows
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
   const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
   const cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
   const cuuint32_t elem_strides[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -179,7 +194,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   CUtensorMap tmc[3], tms[3];
   const int rows[3] = {I, I, H}, Ks[3] = {H, H, I};
   for (int m = 0; m < 3; ++m)
-    if (!make_weight_maps(pool, L, m, rows[m], Ks[m], &tmc[m], &tms[m])) {
+    if (!make_weight_maps(pool, L, m, rows[m], Ks[m], pl.decode ? kDecRows : 128, &tmc[m], &tms[m])) {
       *why = "cuTensorMapEncodeTiled failed for the slot pool";
       return cudaErrorInvalidValue;
     }
@@ -188,7 +203,9 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   int* counts = reinterpret_cast<int*>(w + pl.off_counts);
   int* cnt1 = reinterpret_cast<int*>(w + pl.off_cnt1);
   int* cnt2 = reinterpret_cast<int*>(w + pl.off_cnt2);
-  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(w + pl.off_h);
+  __half* h = reinterpret_cast<__half*>(w + pl.off_h);
+  __half* x16 = reinterpret_cast<__half*>(w + pl.off_x16);
+  float* tokscale = reinterpret_cast<float*>(w + pl.off_tokscale);
   {
   ProfileScope prof(FT_KERNEL_SCHEDULE, s);
   ffn_schedule_kernel<<<1, 1024, 0, s>>>(offsets, slot_table, E, L.num_slots, pl.g1.bn, pl.mt1, pl.g1.splits,
@@ -198,13 +215,23 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
+  {
+    ProfileScope prof(FT_KERNEL_PREP, s);
+    prep_x_kernel<<<(T * k + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(x), perm_src, T * k, k, H,
+                                                  reinterpret_cast<uint4*>(x16), tokscale, counts + 2);
+  }
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
 
   CUtensorMap tm_x, tm_h;
-  if (!make_act_map(x, T, H, 1, &tm_x) || !make_act_map(h, T * k, I, 16, &tm_h)) {
+  const int act_box = pl.decode ? kDecBN : 16;
+  if (!make_act_map(x16, T * k, H, act_box, &tm_x) || !make_act_map(h, T * k, I, act_box, &tm_h)) {
     *why = "cuTensorMapEncodeTiled failed for the activations";
     return cudaErrorInvalidValue;
   }
   FfnParams p1{};
+  p1.tokscale = tokscale;
+  p1.any_scaled = counts + 2;
   p1.perm_src = perm_src;
   p1.k_top = k;
   p1.K = H;
@@ -243,7 +270,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   const int grid2 = int(std::min<long long>(num_sms, pl.max_units2));
 
   if (pl.decode) {
-    err = launch_decode_gemm<2, 2>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    err = launch_decode_gemm<2, 4>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
     if (err == cudaSuccess) err = launch_decode_gemm<1, 4>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   } else {
     err = launch_gemm<2, 128, 3, 4, 4, 1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);

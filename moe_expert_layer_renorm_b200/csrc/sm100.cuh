@@ -22,6 +22,7 @@ enum : int {
   FT_DEV_WAIT_TIMEOUT = 1,
   FT_DEV_NOT_RESIDENT = 2,   // a non-empty expert group maps to slot -1
   FT_DEV_BAD_INDEX = 3,      // an id or slot index outside its range
+  FT_DEV_F16_RANGE = 4,      // an intermediate exceeded the f16 range and was saturated
 };
 
 __device__ __forceinline__ void set_device_status(int code) {
