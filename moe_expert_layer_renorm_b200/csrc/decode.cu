@@ -186,6 +186,9 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
             const uint32_t shi = *reinterpret_cast<const uint16_t*>(sc + r_hi * 16 + 8 * h + 2 * t);
             const uint32_t wlo[4] = {clo.x, clo.y, clo.z, clo.w};
             const uint32_t whi[4] = {chi.x, chi.y, chi.z, chi.w};
+            // the thread's 32 K span two 16-K scale blocks: MMAs 0..3 and 4..7
+            const uint32_t sl2[2] = {e4m3_pair_to_f16x2(slo & 0xFFu), e4m3_pair_to_f16x2(slo >> 8)};
+            const uint32_t sh2[2] = {e4m3_pair_to_f16x2(shi & 0xFFu), e4m3_pair_to_f16x2(shi >> 8)};
 #pragma unroll
             for (int wd = 0; wd < 4; ++wd) {   // word wd: codes of MMAs 2 wd and 2 wd + 1
               // token values for those two MMAs: 16-byte chunk wd of the thread's 64 bytes
@@ -193,8 +196,7 @@ ffn_decode_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_code
               const uint4 b0 = *reinterpret_cast<const uint4*>(bbox + n0 * 128 + ((cb ^ (n0 & 7)) << 4));
               uint4 b1 = make_uint4(0u, 0u, 0u, 0u);
               if (ntiles > 1) b1 = *reinterpret_cast<const uint4*>(bbox + n1 * 128 + ((cb ^ (n1 & 7)) << 4));
-              const uint32_t sl = e4m3_pair_to_f16x2(wd < 2 ? (slo & 0xFFu) : (slo >> 8));
-              const uint32_t sh = e4m3_pair_to_f16x2(wd < 2 ? (shi & 0xFFu) : (shi >> 8));
+              const uint32_t sl = sl2[wd >> 1], sh = sh2[wd >> 1];
               uint32_t qlo[4], qhi[4];
               e2m1x8_to_f16x2(wlo[wd], qlo);
               e2m1x8_to_f16x2(whi[wd], qhi);

@@ -27,19 +27,16 @@ static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Split-K factor: a divisor of the K-stage count (all units of one launch do
 // equal work) that minimises the makespan of the persistent grid, i.e.
-// ceil(units * S / SMs) / (units * S / SMs), with a small charge per split
-// for the partial sums it writes and reduces.
-static int choose_splits(double units_est, int nkw, int num_sms, int* sps_out) {
+// ceil(units * S / SMs) / (units * S / SMs), plus a charge per extra split for
+// the partial sums it writes and reduces (`split_cost`, relative to one
+// unit's own traffic).
+static int choose_splits(double units_est, int nkw, int num_sms, double split_cost, int* sps_out) {
   int best = 1;
   double best_cost = 1e30;
-  if (units_est >= 2.0 * num_sms) {   // enough parallelism: partial sums would only add traffic
-    *sps_out = nkw;
-    return 1;
-  }
   for (int s = 1; s <= std::min(nkw, 16); ++s) {
     if (nkw % s) continue;
     const double work = units_est * s / num_sms;   // waves of equal units
-    const double cost = ceil(work - 1e-9) / work * (1.0 + 0.08 * (s - 1));
+    const double cost = ceil(work - 1e-9) / work * (1.0 + split_cost * (s - 1));
     if (cost < best_cost - 1e-12) { best_cost = cost; best = s; }
   }
   *sps_out = nkw / best;
@@ -76,8 +73,14 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   const double tiles_per_expert2 = std::max(1.0, ceil(mean_rows / pl.g2.bn));
   const double est_tiles1 = std::max(1.0, ceil(distinct) * tiles_per_expert1);
   const double est_tiles2 = std::max(1.0, ceil(distinct) * tiles_per_expert2);
-  pl.g1.splits = choose_splits(est_tiles1 * pl.mt1, pl.nkw1, num_sms, &pl.g1.sps);
-  pl.g2.splits = choose_splits(est_tiles2 * pl.mt2, pl.nkw2, num_sms, &pl.g2.sps);
+  // decode partials are a few token rows per 256 weight rows, but the compute
+  // warps also run the split epilogue (measured: S=4 doubled the gate/up time
+  // at T=64), so splits pay only when they fill idle SMs; prefill
+  // partials are full 128 x 128 fp32 tiles, so prefill splits only to fill the GPU
+  const double split_cost1 = pl.decode ? 0.1 : (est_tiles1 * pl.mt1 >= num_sms ? 1.0 : 0.15);
+  const double split_cost2 = pl.decode ? 0.1 : (est_tiles2 * pl.mt2 >= num_sms ? 1.0 : 0.15);
+  pl.g1.splits = choose_splits(est_tiles1 * pl.mt1, pl.nkw1, num_sms, split_cost1, &pl.g1.sps);
+  pl.g2.splits = choose_splits(est_tiles2 * pl.mt2, pl.nkw2, num_sms, split_cost2, &pl.g2.sps);
   const long long active = std::min<long long>(E, P);
   pl.max_tiles1 = active + P / pl.g1.bn;
   pl.max_tiles2 = active + P / pl.g2.bn;
