@@ -45,7 +45,7 @@ def parse_args():
     ap.add_argument("--workload", default="decode_T64", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--layers", type=int, default=4, help="independent layers the steps rotate over")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-sample-tokens", type=int, default=16)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -119,7 +119,19 @@ class ClockSampler:
 
 # ------------------------------------------------------------ our arm ---
 
-def traffic_record(kernel_src: str, key: str):
+def kernel_source_hash() -> str:
+    """Hash of the sources of the two expert GEMM kernels, the helpers they
+    include and the host code that sizes their launches: a counter taken on
+    other sources no longer describes the launches that run."""
+    d = os.path.join(ROOT, "moe_expert_layer_renorm_b200", "csrc")
+    h = hashlib.sha256()
+    for name in ("sm100.cuh", "ffn.cu", "decode.cu", "ffn_host.cu"):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(key: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel source (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -129,9 +141,50 @@ def traffic_record(kernel_src: str, key: str):
         rec = json.load(f).get(key)
     if not rec:
         return None
-    with open(kernel_src, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:16]
-    return rec["bytes_per_launch"] if rec.get("src_sha256_16") == h else None
+    return rec["bytes_per_launch"] if rec.get("src_sha256_16") == kernel_source_hash() else None
+
+
+L2_BYTES = 126e6
+
+
+def rank_layer_seed(w, rank: int, layer: int) -> int:
+    """Seed of layer `layer` on rank `rank`: every rank draws its own batches
+    and weights (weak scaling over independent problems)."""
+    return inputs.layer_seed(w.seed + 1_000_003 * rank, layer)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a per-rank number over all ranks (the value itself without
+    a process group).  Every rank must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rotation_layers(w, requested: int) -> int:
+    """Independent layers the steps rotate over: at least `requested`, and
+    enough that the weights the other layers read between two visits of a
+    layer (about 3x L2) have evicted that layer's weights from L2."""
+    per_step = inputs.expected_distinct_experts(w.T, w.E, w.k) * bytes_per_expert(w.H, w.I)
+    need = int(np.ceil(3.0 * L2_BYTES / max(per_step, 1.0))) + 1
+    return int(min(64, max(1, requested, need)))
+
+
+def workload_config(w, R: int, S: int, world: int, distinct: float) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    step_mb = distinct * bytes_per_expert(w.H, w.I) / 1e6
+    return {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "H": w.H, "I": w.I,
+            "route": "softmax_renorm" if w.route_mode == 0 else "topk_softmax",
+            "slots": w.slots, "layers_rotated": R, "pool_slots": S,
+            "parallelism": f"dp{world} (independent batches)",
+            "l2": "steps rotate over %d independent layers reading %.0f MB of expert weights per step; "
+                  "a layer's weights come back after %.0f MB of other layers' (L2 is 126 MB)"
+                  % (R, step_mb, (R - 1) * step_mb)}
 
 
 def run_ours(args):
@@ -149,22 +202,26 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     w = inputs.WORKLOADS[args.workload]
-    R = max(1, args.layers)
+    R = rotation_layers(w, args.layers)
     T = w.T
-    # per-rank, per-layer independent inputs
+    # per-rank, per-layer independent inputs; the R layers' experts share one
+    # slot pool (disjoint slots, scattered over the pool when the workload's
+    # slots are permuted), as the layers of a model share an expert cache
+    S = max(w.slots, R * w.E)
+    order = np.random.default_rng([w.seed, rank, 9]).permutation(S) if w.permuted_slots else np.arange(S)
+    pool = ExpertPool(w.H, w.I, S, device=dev)
     layers = []
     for l in range(R):
-        s = inputs.layer_seed(w.seed + 1_000_003 * rank, l)
+        s = rank_layer_seed(w, rank, l)
         li = inputs.make_layer_inputs(inputs.custom_workload(w, seed=s), 0)
-        st = li.slot_table
-        pool = ExpertPool(w.H, w.I, w.slots, device=dev)
+        st = order[l * w.E:(l + 1) * w.E].astype(np.int32)
         for e in range(w.E):
             for mat in range(3):
                 N, K = pool.shape(mat)
                 pool.pack_into(int(st[e]), mat, inputs.make_weight_fp32_torch(N, K, s, e, mat, dev))
         x = torch.from_numpy(li.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
         lg = torch.from_numpy(li.logits).to(dev)
-        layers.append(dict(li=li, pool=pool, st=torch.from_numpy(st).to(dev), x=x, lg=lg, seed=s))
+        layers.append(dict(li=li, pool=pool, st_host=st, st=torch.from_numpy(st).to(dev), x=x, lg=lg, seed=s))
     torch.cuda.synchronize()
     layer = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev)
     stream = torch.cuda.Stream(device=dev)
@@ -213,10 +270,7 @@ def run_ours(args):
                 fn(i)
             b.record(stream)
         stream.synchronize()
-        t = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(a.elapsed_time(b), dev)
 
     # -------- timed region 1: graph replays, device-resident inputs --------
     clocks = ClockSampler(local)
@@ -282,8 +336,7 @@ def run_ours(args):
     else:
         alg_bytes = mean_distinct * (w.H * w.I // 2 + w.H * w.I // 16 + 4) + P * w.I * 2 + P * w.H * 4
         alg_flops = 2.0 * w.H * w.I * P
-    src = os.path.join(ROOT, "moe_expert_layer_renorm_b200", "csrc", "ffn.cu")
-    traffic = traffic_record(src, f"{dom_name}:{args.workload}")
+    traffic = traffic_record(f"{dom_name}:{args.workload}")
     if decode_like:
         achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
@@ -291,7 +344,11 @@ def run_ours(args):
                 "launch_ms": round(dom_ms, 5), "algorithmic_bytes": int(alg_bytes), "peak_source": peak_src}
     else:
         achieved = alg_flops / (dom_ms * 1e-3) / 1e12
-        peak = bf16_sus
+        # the burst GEMM peak while the SMs held their maximum clock through the
+        # timed region, the sustained (power-capped) one otherwise
+        full_clock = bool(clk.get("sm_mhz") and clk.get("sm_max_mhz") and clk["sm_mhz"] >= 0.95 * clk["sm_max_mhz"])
+        peak = bf16 if full_clock else bf16_sus
+        peak_src = f"{peak_src} ({'burst' if full_clock else 'sustained'} bf16 GEMM)"
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": dom_name,
                 "launch_ms": round(dom_ms, 5), "algorithmic_flops": alg_flops, "peak_source": peak_src}
@@ -314,13 +371,9 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 weights, bf16 activations, fp32 accumulate",
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 weights, f16 MMA operands, fp32 accumulate",
         "data": "synthetic (seeded N(0,1) activations, N(0,sigma) logits, N(0,0.02) weights packed to NVFP4)",
-        "config": {"workload": args.workload, "T": T, "E": w.E, "k": w.k, "H": w.H, "I": w.I,
-                   "route": "softmax_renorm" if w.route_mode == 0 else "topk_softmax",
-                   "slots": w.slots, "layers_rotated": R, "parallelism": f"dp{world} (independent batches)",
-                   "l2": "steps rotate over %d layers; each step reads %.0f MB of expert weights > 126 MB L2"
-                         % (R, mean_distinct * bytes_per_expert(w.H, w.I) / 1e6)},
+        "config": workload_config(w, R, S, world, mean_distinct),
         "layer": {"distinct_experts": round(mean_distinct, 2), "weight_GBps": round(layer_gbs, 1),
                   "TFLOPs": round(layer_tflops, 2), "hbm_frac_of_measured": round(layer_gbs / hbm, 4)},
         "roofline": roof,
@@ -344,7 +397,7 @@ def cpu_baseline(L, w, T, n_tokens):
 
     li = L["li"]
     pool = L["pool"]
-    st = li.slot_table
+    st = L["st_host"]
     n = min(T, n_tokens)
     ids, _ = M.route(li.logits[:n], w.k)
     exps = {}
@@ -367,6 +420,9 @@ def cpu_baseline(L, w, T, n_tokens):
 
 # ------------------------------------------------------ reference arm ---
 
+REFERENCE_BUDGET_S = 120.0
+
+
 def run_reference(args):
     """The CPU oracle timed on the host cores, on this workload's metric."""
     rank, world, _ = dist_env()
@@ -378,6 +434,7 @@ def run_reference(args):
     from oracle import nvfp4
 
     w = inputs.WORKLOADS[args.workload]
+    R = rotation_layers(w, args.layers)
     li = inputs.make_layer_inputs(w, 0)
     s = inputs.layer_seed(w.seed, 0)
     n = min(w.T, args.cpu_sample_tokens)
@@ -400,6 +457,12 @@ def run_reference(args):
         M.moe_layer(li.x_bits[tok], li.logits[tok], w.k, exps, keep_out_perm=False)
         return time.perf_counter() - t0
 
+    # size each step's sample so that warm-up and timed steps together take
+    # about REFERENCE_BUDGET_S of host time
+    n = min(n, 2)
+    per_token = step(0) / n
+    n = int(max(1, min(w.T, args.cpu_sample_tokens,
+                       REFERENCE_BUDGET_S / max(1, args.steps + args.warmup) / max(per_token, 1e-9))))
     for i in range(args.warmup):
         step(i)
     times = [step(args.warmup + i) for i in range(args.steps)]
@@ -410,7 +473,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": args.workload, "T": w.T, "E": w.E, "k": w.k, "H": w.H, "I": w.I},
+        "data": "synthetic", "config": workload_config(w, R, max(w.slots, R * w.E), world,
+                                                        inputs.expected_distinct_experts(w.T, w.E, w.k)),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": f"{n} tokens of one {w.name} layer per step"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
