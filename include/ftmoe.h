@@ -135,6 +135,28 @@ FT_API int ft_moe_permute(const int32_t* topk_ids, int T, int k, int E,
 FT_API size_t ft_moe_permute_workspace_size(int T, int k, int E);
 
 /*
+ * ft_moe_permute without a workspace argument and without allocating.  The
+ * pages have no counterpart of this call: it is an interface convenience.
+ * Output is identical, bit for bit, to ft_moe_permute's.
+ *
+ * It is meant for callers that cannot draw device memory when they call:
+ * a host program with no device allocator, or a runtime whose device memory
+ * is all partitioned at start-up.  The per-chunk counts go to a fixed
+ * 256 KiB array inside this library, which limits inputs to
+ * ceil(T*k / 1024) * E <= 65536 (always met when T*k <= 1024); larger inputs
+ * return FT_ERR_INVALID_ARG and launch nothing.  The array needs no zeroing.
+ *
+ * The first call with a given device current looks up that device's copy of
+ * the array; make it before any stream capture.  Calls on one device share
+ * the array: two calls that can overlap in time (different streams, or
+ * different host threads) race and give wrong rows, so order them.
+ * Arguments are those of ft_moe_permute minus ws and ws_bytes.
+ */
+FT_API int ft_moe_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
+                   int32_t* expert_offsets, int32_t* perm_src, int32_t* pair_to_row,
+                   ft_stream_t stream);
+
+/*
  * Expert FFN over the permuted rows.  For row r of group e (token
  * t = perm_src[r] / k), with the expert's tensors at
  * slot_pool + slot_table[e] * layout->slot_bytes:

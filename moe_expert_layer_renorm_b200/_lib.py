@@ -69,6 +69,7 @@ _SIGS = {
     "ft_moe_permute": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                c_void_p]),
     "ft_moe_permute_workspace_size": (c_size_t, [c_int, c_int, c_int]),
+    "ft_moe_permute_noalloc": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "ft_moe_ffn_nvfp4": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
                                  c_void_p, POINTER(SlotLayout), c_void_p, c_void_p, c_size_t, c_void_p]),
     "ft_moe_ffn_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
@@ -127,6 +128,12 @@ def permute_workspace_size(T, k, E) -> int:
 
 def permute(ids, T, k, E, offsets, perm_src, pair_to_row, ws, ws_bytes, stream) -> None:
     check(lib().ft_moe_permute(ids, T, k, E, offsets, perm_src, pair_to_row, ws, ws_bytes, stream))
+
+
+def permute_noalloc(ids, T, k, E, offsets, perm_src, pair_to_row, stream) -> None:
+    """ft_moe_permute without a workspace: for callers that cannot allocate
+    device memory at call time (limits and sharing rules in the C header)."""
+    check(lib().ft_moe_permute_noalloc(ids, T, k, E, offsets, perm_src, pair_to_row, stream))
 
 
 def ffn_workspace_size(T, H, I, E, k) -> int:

@@ -15,4 +15,5 @@
 #include "decode.cu"
 #include "ffn_host.cu"
 #include "api.cu"
+#include "permute_noalloc.cu"
 #include "slots.cpp"
