@@ -292,7 +292,8 @@ enum {
   FT_KERNEL_COMBINE = 5,
   FT_KERNEL_PACK = 6,
   FT_KERNEL_PREP = 7,         /* activations to f16 (inside ft_moe_ffn_nvfp4) */
-  FT_KERNEL_KINDS = 8,
+  FT_KERNEL_FFN_DECODE = 8,   /* decode variant: gate/up + SwiGLU + down in one launch */
+  FT_KERNEL_KINDS = 9,
 };
 
 typedef struct {

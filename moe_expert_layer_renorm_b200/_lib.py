@@ -52,11 +52,12 @@ class SlotLayout(ctypes.Structure):
     ]
 
 
-FT_KERNEL_NAMES = ("route", "permute", "schedule", "gemm_gate_up", "gemm_down", "combine", "pack", "prep_x")
+FT_KERNEL_NAMES = ("route", "permute", "schedule", "gemm_gate_up", "gemm_down", "combine", "pack", "prep_x",
+                   "ffn_decode")
 
 
 class Profile(ctypes.Structure):
-    _fields_ = [("launches", c_int64 * 8), ("timed", c_int64 * 8), ("total_ms", ctypes.c_double * 8)]
+    _fields_ = [("launches", c_int64 * 9), ("timed", c_int64 * 9), ("total_ms", ctypes.c_double * 9)]
 
 
 class SlotStats(ctypes.Structure):

@@ -111,8 +111,9 @@ extern "C" int ft_moe_ffn_nvfp4(const void* x, int T, int H, int I, int E, int k
   if (T == 0) return FT_OK;
   if (!x || !perm_src || !expert_offsets || !slot_table || !slot_pool || !layout || !out_perm || !ws)
     return fail(FT_ERR_INVALID_ARG, "ft_moe_ffn_nvfp4: null pointer");
-  if (layout->H != H || layout->I != I || layout->num_slots < 1 || layout->slot_bytes % 256)
-    return fail(FT_ERR_INVALID_ARG, "ft_moe_ffn_nvfp4: layout does not match H, I");
+  if (layout->H != H || layout->I != I || layout->num_slots < 1 || layout->num_slots > (1 << 21) ||
+      layout->slot_bytes % 256)
+    return fail(FT_ERR_INVALID_ARG, "ft_moe_ffn_nvfp4: layout does not match H, I (or has more than 2^21 slots)");
   if ((reinterpret_cast<uintptr_t>(slot_pool) & 255) || (reinterpret_cast<uintptr_t>(ws) & 255) ||
       (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(out_perm) & 15))
     return fail(FT_ERR_INVALID_ARG, "ft_moe_ffn_nvfp4: misaligned pointer");

@@ -53,7 +53,7 @@ struct FfnParams {
   int nkc;                    // K / kKC
   int splits;                 // split-K factor
   int stages_per_split;
-  const int4* units;          // {expert, m_tile, row_begin, n_rows | split << 16}
+  const int4* units;          // {expert | slot << 10, m_tile, row_begin, n_rows | split << 16}
   const int* num_units;
   const int32_t* slot_table;
   const uint8_t* pool;
@@ -228,7 +228,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
 
   auto unit_range = [&](int u, int& e, int& mt, int& rb, int& nr, int& ws0, int& ws1, int& kc0, int& kc1) {
     const int4 d = p.units[u];
-    e = d.x; mt = d.y; rb = d.z; nr = d.w & 0xFFFF;
+    e = d.x & 1023; mt = d.y; rb = d.z; nr = d.w & 0xFFFF;
     const int split = d.w >> 16;
     ws0 = split * p.stages_per_split;
     ws1 = min(p.nkw, ws0 + p.stages_per_split);
@@ -537,15 +537,16 @@ __device__ int block_exclusive_scan(int v, int* smem_warp_sums);
 __global__ void __launch_bounds__(1024) ffn_schedule_kernel(
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ slot_table, int E, int num_slots,
     int bn1, int mt1, int s1, int bn2, int mt2, int s2, int4* __restrict__ units1, int4* __restrict__ units2,
-    int* __restrict__ counts, int* __restrict__ counters1, int ncnt1, int* __restrict__ counters2, int ncnt2) {
+    int* __restrict__ counts, int* __restrict__ counters1, int ncnt1, int* __restrict__ counters2, int ncnt2,
+    int* __restrict__ tile_done, int ndone) {
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
-  int n = 0, rb = 0;
+  int n = 0, rb = 0, slot = 0;
   if (e < E) {
     rb = offsets[e];
     n = offsets[e + 1] - rb;
     if (n > 0) {
-      const int slot = slot_table[e];
+      slot = slot_table[e];
       if (slot < 0) { set_device_status(FT_DEV_NOT_RESIDENT); n = 0; }
       else if (slot >= num_slots) { set_device_status(FT_DEV_BAD_INDEX); n = 0; }
     }
@@ -556,17 +557,21 @@ __global__ void __launch_bounds__(1024) ffn_schedule_kernel(
   for (int t = 0; t < t1; ++t)
     for (int m = 0; m < mt1; ++m)
       for (int s = 0; s < s1; ++s)
-        units1[((ex1 + t) * mt1 + m) * s1 + s] = make_int4(e, m, rb + t * bn1, min(bn1, n - t * bn1) | (s << 16));
+        units1[((ex1 + t) * mt1 + m) * s1 + s] =
+            make_int4(e | (slot << 10), m, rb + t * bn1, min(bn1, n - t * bn1) | (s << 16));
   for (int t = 0; t < t2; ++t)
     for (int m = 0; m < mt2; ++m)
       for (int s = 0; s < s2; ++s)
-        units2[((ex2 + t) * mt2 + m) * s2 + s] = make_int4(e, m, rb + t * bn2, min(bn2, n - t * bn2) | (s << 16));
+        units2[((ex2 + t) * mt2 + m) * s2 + s] =
+            make_int4(e | (slot << 10), m, rb + t * bn2, min(bn2, n - t * bn2) | (s << 16));
   if (e == blockDim.x - 1) {
     counts[0] = (ex1 + t1) * mt1 * s1;
     counts[1] = (ex2 + t2) * mt2 * s2;
   }
+  if (threadIdx.x == 0) { counts[2] = 0; counts[3] = 0; }   // any token prescaled; unit queue
   for (int i = threadIdx.x; i < ncnt1; i += blockDim.x) counters1[i] = 0;
   for (int i = threadIdx.x; i < ncnt2; i += blockDim.x) counters2[i] = 0;
+  for (int i = threadIdx.x; i < ndone; i += blockDim.x) tile_done[i] = 0;
 }
 
 }  // namespace ftmoe

@@ -17,8 +17,8 @@ struct FfnPlan {
   int mt1, mt2, nkw1, nkw2, nkc1, nkc2;
   long long max_tiles1, max_tiles2;
   // workspace layout (byte offsets)
-  size_t off_h, off_x16, off_tokscale, off_units1, off_units2, off_counts, off_cnt1, off_cnt2, off_part1, off_part2,
-      total;
+  size_t off_h, off_x16, off_tokscale, off_units1, off_units2, off_counts, off_cnt1, off_cnt2, off_done, off_part1,
+      off_part2, total;
   long long max_units1, max_units2;
   int cnt_per;
 };
@@ -43,10 +43,24 @@ static int choose_splits(double units_est, int nkw, int num_sms, double split_co
   return best;
 }
 
+// Decode split-K: the smallest divisor of the K-stage count that gives every
+// SM a unit (a dynamic queue balances the rest, so waves do not matter).
+static int decode_splits(double units_est, int nkw, int num_sms, int* sps_out) {
+  int best = 1;
+  for (int s = 1; s <= std::min(nkw, 16); ++s) {
+    if (nkw % s) continue;
+    best = s;
+    if (units_est * s >= num_sms) break;
+  }
+  *sps_out = nkw / best;
+  return best;
+}
+
 // Variant choice: groups of a few token rows (mean rows per active expert
 // <= kDecodeMeanRows) are bound by the weight bytes and take the
-// weight-streaming decode kernel (256-row tiles, 16-row token units); larger
-// groups take the tcgen05 kernel (128-row tiles, 128-row token units).
+// weight-streaming decode kernel (both GEMMs in one launch, 16-row token
+// units); larger groups take the tcgen05 kernel (128-row tiles, 128-row
+// token units).
 constexpr double kDecodeMeanRows = 16.0;
 
 static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
@@ -55,9 +69,8 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   const double distinct = E * (1.0 - pow(1.0 - double(k) / E, double(T)));
   const double mean_rows = distinct > 0 ? double(P) / distinct : 0.0;
   pl.decode = mean_rows <= kDecodeMeanRows;
-  const int tile_rows = pl.decode ? kDecRows : 128;
-  pl.mt1 = (I + tile_rows - 1) / tile_rows;
-  pl.mt2 = (H + tile_rows - 1) / tile_rows;
+  pl.mt1 = (I + (pl.decode ? kDecFeat1 : 128) - 1) / (pl.decode ? kDecFeat1 : 128);
+  pl.mt2 = (H + (pl.decode ? kDecRows : 128) - 1) / (pl.decode ? kDecRows : 128);
   pl.nkw1 = (H + kKW - 1) / kKW;
   pl.nkw2 = (I + kKW - 1) / kKW;
   pl.nkc1 = H / kKC;
@@ -73,14 +86,16 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   const double tiles_per_expert2 = std::max(1.0, ceil(mean_rows / pl.g2.bn));
   const double est_tiles1 = std::max(1.0, ceil(distinct) * tiles_per_expert1);
   const double est_tiles2 = std::max(1.0, ceil(distinct) * tiles_per_expert2);
-  // decode partials are a few token rows per 256 weight rows, but the compute
-  // warps also run the split epilogue (measured: S=4 doubled the gate/up time
-  // at T=64), so splits pay only when they fill idle SMs; prefill
-  // partials are full 128 x 128 fp32 tiles, so prefill splits only to fill the GPU
-  const double split_cost1 = pl.decode ? 0.1 : (est_tiles1 * pl.mt1 >= num_sms ? 1.0 : 0.15);
-  const double split_cost2 = pl.decode ? 0.1 : (est_tiles2 * pl.mt2 >= num_sms ? 1.0 : 0.15);
-  pl.g1.splits = choose_splits(est_tiles1 * pl.mt1, pl.nkw1, num_sms, split_cost1, &pl.g1.sps);
-  pl.g2.splits = choose_splits(est_tiles2 * pl.mt2, pl.nkw2, num_sms, split_cost2, &pl.g2.sps);
+  if (pl.decode) {
+    pl.g1.splits = decode_splits(est_tiles1 * pl.mt1, pl.nkw1, num_sms, &pl.g1.sps);
+    pl.g2.splits = decode_splits(est_tiles2 * pl.mt2, pl.nkw2, num_sms, &pl.g2.sps);
+  } else {
+    // prefill partials are full 128 x 128 fp32 tiles: split only to fill the GPU
+    const double split_cost1 = est_tiles1 * pl.mt1 >= num_sms ? 1.0 : 0.15;
+    const double split_cost2 = est_tiles2 * pl.mt2 >= num_sms ? 1.0 : 0.15;
+    pl.g1.splits = choose_splits(est_tiles1 * pl.mt1, pl.nkw1, num_sms, split_cost1, &pl.g1.sps);
+    pl.g2.splits = choose_splits(est_tiles2 * pl.mt2, pl.nkw2, num_sms, split_cost2, &pl.g2.sps);
+  }
   const long long active = std::min<long long>(E, P);
   pl.max_tiles1 = active + P / pl.g1.bn;
   pl.max_tiles2 = active + P / pl.g2.bn;
@@ -88,17 +103,18 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   pl.max_units2 = pl.max_tiles2 * pl.mt2 * pl.g2.splits;
   // split-K counters per (tile, m-tile): one per epilogue warp of the kernel
   const int cnt_per = pl.decode ? 16 : 4;
-  const size_t part_unit1 = pl.decode ? size_t(2) * kDecBN * kDecRows * 4 : size_t(2) * 128 * pl.g1.bn * 4;
-  const size_t part_unit2 = pl.decode ? size_t(1) * kDecBN * kDecRows * 4 : size_t(1) * 128 * pl.g2.bn * 4;
+  const size_t part_unit1 = pl.decode ? size_t(kDecPartialBytes) : size_t(2) * 128 * pl.g1.bn * 4;
+  const size_t part_unit2 = pl.decode ? size_t(kDecPartialBytes) : size_t(1) * 128 * pl.g2.bn * 4;
   size_t o = 0;
   pl.off_h = o;       o = align256(o + size_t(P) * I * 2);
   pl.off_x16 = o;     o = align256(o + size_t(P) * H * 2);   // f16 activations, permuted rows
   pl.off_tokscale = o; o = align256(o + size_t(T) * 4);
   pl.off_units1 = o;  o = align256(o + size_t(pl.max_units1) * 16);
   pl.off_units2 = o;  o = align256(o + size_t(pl.max_units2) * 16);
-  pl.off_counts = o;  o = align256(o + 16);   // [0] units of GEMM1, [1] of GEMM2, [2] any token prescaled
+  pl.off_counts = o;  o = align256(o + 16);   // [0] units of GEMM1, [1] of GEMM2, [2] any token prescaled, [3] queue
   pl.off_cnt1 = o;    o = align256(o + size_t(pl.max_tiles1 * pl.mt1) * cnt_per * 4);
   pl.off_cnt2 = o;    o = align256(o + size_t(pl.max_tiles2 * pl.mt2) * cnt_per * 4);
+  pl.off_done = o;    o = align256(o + size_t(pl.max_tiles1) * 4);   // decode: h published per token tile
   pl.off_part1 = o;
   if (pl.g1.splits > 1) o = align256(o + size_t(pl.max_units1) * part_unit1);
   pl.off_part2 = o;
@@ -197,7 +213,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   CUtensorMap tmc[3], tms[3];
   const int rows[3] = {I, I, H}, Ks[3] = {H, H, I};
   for (int m = 0; m < 3; ++m)
-    if (!make_weight_maps(pool, L, m, rows[m], Ks[m], pl.decode ? kDecRows : 128, &tmc[m], &tms[m])) {
+    if (!make_weight_maps(pool, L, m, rows[m], Ks[m], 128, &tmc[m], &tms[m])) {
       *why = "cuTensorMapEncodeTiled failed for the slot pool";
       return cudaErrorInvalidValue;
     }
@@ -214,7 +230,8 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   ffn_schedule_kernel<<<1, 1024, 0, s>>>(offsets, slot_table, E, L.num_slots, pl.g1.bn, pl.mt1, pl.g1.splits,
                                          pl.g2.bn, pl.mt2, pl.g2.splits, units1, units2, counts, cnt1,
                                          int(pl.max_tiles1 * pl.mt1 * pl.cnt_per), cnt2,
-                                         int(pl.max_tiles2 * pl.mt2 * pl.cnt_per));
+                                         int(pl.max_tiles2 * pl.mt2 * pl.cnt_per),
+                                         reinterpret_cast<int*>(w + pl.off_done), pl.decode ? int(pl.max_tiles1) : 0);
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -273,8 +290,15 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   const int grid2 = int(std::min<long long>(num_sms, pl.max_units2));
 
   if (pl.decode) {
-    err = launch_decode_gemm<2, 4>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
-    if (err == cudaSuccess) err = launch_decode_gemm<1, 4>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
+    DecodeParams dp{};
+    dp.g[0] = p1;
+    dp.g[1] = p2;
+    dp.queue = counts + 3;
+    dp.tile_done = reinterpret_cast<int*>(w + pl.off_done);
+    dp.mt1 = pl.mt1;
+    dp.mt2 = pl.mt2;
+    const int grid = int(std::min<long long>(num_sms, pl.max_units1 + pl.max_units2));
+    err = launch_decode(dp, grid, tmc, tms, tm_x, tm_h, s);
   } else {
     err = launch_gemm<2, 128, 3, 4, 4, 1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
     if (err == cudaSuccess) err = launch_gemm<1, 128, 3, 6, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);

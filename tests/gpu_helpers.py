@@ -63,6 +63,10 @@ def run_gpu(w: inputs.Workload, T: Optional[int] = None, layer: int = 0, pool=No
     logits = torch.from_numpy(li.logits).cuda()
     st = torch.from_numpy(np.asarray(slot_table, dtype=np.int32)).cuda()
     lay = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode)
+    # NaN in every intermediate the library writes before reading: an element
+    # read before it is written (a missed dependency) shows up in y
+    lay.ffn_ws.fill_(0xFF)
+    lay.out_perm.fill_(float("nan"))
     from moe_expert_layer_renorm_b200 import _lib
     _lib.device_status(clear=True)
     y = lay.forward(x, logits, st, pool)
