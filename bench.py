@@ -396,32 +396,39 @@ def run_ours(args):
     print(json.dumps(line))
 
 
-def cpu_baseline(L, w, T, n_tokens):
-    """The oracle (as it stands) on a bounded sample of the same layer."""
-    from threadpoolctl import threadpool_info
+def oracle_threads() -> int:
+    """Host threads the C++ oracle runs on (its OpenMP default)."""
+    v = os.environ.get("OMP_NUM_THREADS", "")
+    return int(v) if v.isdigit() and int(v) > 0 else (os.cpu_count() or 1)
 
-    from oracle import moe_layer as M
+
+def cpu_baseline(L, w, T, n_tokens):
+    """The C++ oracle (as it stands) on a bounded sample of the same layer:
+    the first n tokens, repeated until about 10 s of host time."""
+    from oracle import cpp
 
     li = L["li"]
     pool = L["pool"]
     st = L["st_host"]
     n = min(T, n_tokens)
-    ids, _ = M.route(li.logits[:n], w.k)
-    exps = {}
-    for e in sorted(set(int(v) for v in ids.reshape(-1))):
-        mats = []
-        for mat in range(3):
-            c, sc, g = pool.tensor_bytes(int(st[e]), mat)
-            N, K = pool.shape(mat)
-            mats.append(M.Nvfp4Tensor(c, sc, g, N, K))
-        exps[e] = M.Expert(*mats)
-    t0 = time.perf_counter()
-    M.moe_layer(li.x_bits[:n], li.logits[:n], w.k, exps, keep_out_perm=False)
-    dt = time.perf_counter() - t0
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} tokens of one {w.name} layer (route, permute, NVFP4 decode of the "
-                      f"{len(exps)} experts they select, fp64 SwiGLU FFN, combine); {dt:.2f} s",
+    ids, _ = cpp.route(li.logits[:n], w.k)
+    need = sorted(set(int(v) for v in ids.reshape(-1)))
+    buf = np.zeros(len(need) * pool.slot_bytes, np.uint8)     # the selected experts' slots, on the host
+    table = np.full(w.E, -1, np.int32)
+    for i, e in enumerate(need):
+        buf[i * pool.slot_bytes:(i + 1) * pool.slot_bytes] = pool.slot_view(int(st[e])).cpu().numpy()
+        table[e] = i
+    Lo = pool.layout
+    reps, dt = 0, 0.0
+    while dt < 10.0 and reps < 50:
+        t0 = time.perf_counter()
+        cpp.moe_layer(li.x_bits, li.logits, w.k, table, buf, pool.slot_bytes, list(Lo.codes_off),
+                      list(Lo.scales_off), list(Lo.global_off), list(Lo.ld_scale), w.H, w.I, tokens=np.arange(n))
+        dt += time.perf_counter() - t0
+        reps += 1
+    return {"value": round(n * reps / dt, 3), "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{n} tokens of one {w.name} layer x {reps} (C++ oracle: route, NVFP4 decode from the "
+                      f"bytes of the {len(need)} experts they select, fp64 SwiGLU FFN, combine); {dt:.2f} s",
             "host_cpus": os.cpu_count()}
 
 
@@ -430,52 +437,74 @@ def cpu_baseline(L, w, T, n_tokens):
 REFERENCE_BUDGET_S = 120.0
 
 
+def reference_layout(H: int, I: int) -> dict:
+    """The slot layout of the library's C header (ft_nvfp4_slot_layout) from its
+    documented definition, for the reference arm, which loads no library."""
+    a256 = lambda v: (v + 255) // 256 * 256
+    L = {"codes_off": [], "scales_off": [], "ld_scale": []}
+    off = 0
+    for N, K in ((I, H), (I, H), (H, I)):
+        ld = (K // 16 + 15) // 16 * 16
+        L["ld_scale"].append(ld)
+        L["codes_off"].append(off)
+        off = a256(off + N * K // 2)
+        L["scales_off"].append(off)
+        off = a256(off + N * ld)
+    L["global_off"] = [off + 4 * m for m in range(3)]
+    L["slot_bytes"] = a256(off + 12)
+    return L
+
+
 def run_reference(args):
-    """The CPU oracle timed on the host cores, on this workload's metric."""
+    """The C++ oracle timed on the host cores, on this workload's metric."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    from threadpoolctl import threadpool_info
-
-    from oracle import moe_layer as M
-    from oracle import nvfp4
+    from oracle import cpp
 
     w = inputs.WORKLOADS[args.workload]
     R = rotation_layers(w, args.layers)
     li = inputs.make_layer_inputs(w, 0)
     s = inputs.layer_seed(w.seed, 0)
-    n = min(w.T, args.cpu_sample_tokens)
-    cache = {}
+    Lo = reference_layout(w.H, w.I)
+    slots = {}
 
-    def expert(e):
-        if e not in cache:
-            mats = []
+    def slot_bytes_of(e):
+        """Expert e packed by the oracle into one slot of the layout (untimed)."""
+        if e not in slots:
+            b = np.zeros(Lo["slot_bytes"], np.uint8)
             for mat, (N, K) in enumerate(((w.I, w.H), (w.I, w.H), (w.H, w.I))):
-                c, sc, g = nvfp4.pack(inputs.make_weight_fp32_host(N, K, s, e, mat))
-                mats.append(M.Nvfp4Tensor(c, sc, g, N, K))
-            cache[e] = M.Expert(*mats)
-        return cache[e]
+                c, sc, g = cpp.pack(inputs.make_weight_fp32_host(N, K, s, e, mat), Lo["ld_scale"][mat])
+                b[Lo["codes_off"][mat]:Lo["codes_off"][mat] + c.size] = c.reshape(-1)
+                b[Lo["scales_off"][mat]:Lo["scales_off"][mat] + sc.size] = sc.reshape(-1)
+                b[Lo["global_off"][mat]:Lo["global_off"][mat] + 4] = np.frombuffer(np.float32(g).tobytes(), np.uint8)
+            slots[e] = b
+        return slots[e]
 
-    def step(i):
+    def step(i, n):
         tok = (np.arange(n) + i * n) % w.T
-        ids, _ = M.route(li.logits[tok], w.k)
-        exps = {int(e): expert(int(e)) for e in np.unique(ids)}
+        ids, _ = cpp.route(li.logits[tok], w.k)
+        need = sorted(set(int(v) for v in ids.reshape(-1)))
+        buf = np.concatenate([slot_bytes_of(e) for e in need])
+        table = np.full(w.E, -1, np.int32)
+        table[need] = np.arange(len(need), dtype=np.int32)
         t0 = time.perf_counter()
-        M.moe_layer(li.x_bits[tok], li.logits[tok], w.k, exps, keep_out_perm=False)
+        cpp.moe_layer(li.x_bits, li.logits, w.k, table, buf, Lo["slot_bytes"], Lo["codes_off"], Lo["scales_off"],
+                      Lo["global_off"], Lo["ld_scale"], w.H, w.I, tokens=tok)
         return time.perf_counter() - t0
 
     # size each step's sample so that warm-up and timed steps together take
     # about REFERENCE_BUDGET_S of host time
-    n = min(n, 2)
-    per_token = step(0) / n
+    n0 = min(w.T, 2)
+    per_token = step(0, n0) / n0
     n = int(max(1, min(w.T, args.cpu_sample_tokens,
                        REFERENCE_BUDGET_S / max(1, args.steps + args.warmup) / max(per_token, 1e-9))))
     for i in range(args.warmup):
-        step(i)
-    times = [step(args.warmup + i) for i in range(args.steps)]
+        step(i, n)
+    times = [step(args.warmup + i, n) for i in range(args.steps)]
     total = sum(times)
     value = n * args.steps / total
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    threads = oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),

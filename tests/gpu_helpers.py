@@ -91,17 +91,37 @@ def check_routing(run: GpuRun, k: int):
     return ids
 
 
+def host_pool(pool: ExpertPool, slot_table: np.ndarray, experts):
+    """The slots of the given experts copied to the host, packed densely, and
+    the slot table that points into that copy (-1 for the other experts)."""
+    need = sorted(set(int(v) for v in experts))
+    L = pool.layout
+    buf = np.zeros(max(1, len(need)) * pool.slot_bytes, np.uint8)
+    table = np.full(len(slot_table), -1, np.int32)
+    for i, e in enumerate(need):
+        buf[i * pool.slot_bytes:(i + 1) * pool.slot_bytes] = pool.slot_view(int(slot_table[e])).cpu().numpy()
+        table[e] = i
+    return buf, table, L
+
+
+def reference_y(run: GpuRun, k: int, tok: np.ndarray) -> np.ndarray:
+    """The C++ oracle's y for the tokens `tok`, from the packed bytes in the pool."""
+    from oracle import cpp
+    ids = run.layer.ids.cpu().numpy()
+    buf, table, L = host_pool(run.pool, run.slot_table, ids[tok].reshape(-1))
+    H, I = run.pool.H, run.pool.I
+    return cpp.moe_layer(run.x_bits, run.logits, k, table, buf, run.pool.slot_bytes, list(L.codes_off),
+                         list(L.scales_off), list(L.global_off), list(L.ld_scale), H, I, tokens=tok)
+
+
 def check_output(run: GpuRun, k: int, tokens: Optional[Sequence[int]] = None):
     """y within 1e-2 * rms(y_ref) + 1e-3 element-wise (rms over the evaluated tokens)."""
-    ids = run.layer.ids.cpu().numpy()
     T = run.x_bits.shape[0]
     tok = np.arange(T) if tokens is None else np.asarray(tokens)
-    exps = oracle_experts(run.pool, run.slot_table, ids[tok].reshape(-1))
-    ref = M.moe_layer(run.x_bits, run.logits, k, exps, tokens=None if tokens is None else tok,
-                      keep_out_perm=False)
+    ref_y = reference_y(run, k, tok)
     y = run.y[tok]
-    tol = M.tolerance(ref.y)
-    err = np.abs(y - ref.y)
+    tol = M.tolerance(ref_y)
+    err = np.abs(y - ref_y)
     worst = float(err.max()) if err.size else 0.0
-    assert np.all(err <= tol), f"max |err| {worst:.3g} > tol {tol:.3g} (rms {np.sqrt(np.mean(ref.y ** 2)):.3g})"
+    assert np.all(err <= tol), f"max |err| {worst:.3g} > tol {tol:.3g} (rms {np.sqrt(np.mean(ref_y ** 2)):.3g})"
     return worst, tol

@@ -98,3 +98,13 @@ def test_workspace_queries(L):
     big = _lib.ffn_workspace_size(4096, 2048, 768, 128, 8)
     assert small > 16 * 2 * 512 * 2 and big > 4096 * 8 * 768 * 2
     assert _lib.ffn_workspace_size(0, 2048, 768, 128, 8) == 0
+
+
+@pytest.mark.parametrize("H,I", [(256, 512), (2048, 768), (2880, 2880), (320, 448)])
+def test_reference_layout_matches_library(H, I):
+    import bench
+    ref = bench.reference_layout(H, I)
+    L = _lib.slot_layout(H, I, 3)
+    assert list(L.ld_scale) == ref["ld_scale"] and list(L.codes_off) == ref["codes_off"]
+    assert list(L.scales_off) == ref["scales_off"] and list(L.global_off) == ref["global_off"]
+    assert L.slot_bytes == ref["slot_bytes"]
