@@ -23,25 +23,23 @@
 // the wait always ends.  The down unit's weights stream in meanwhile.
 //
 // CTA (18 warps):
-//   warps 0-15  compute, as 4 row groups x 4 K groups: warp w owns rows
-//               64 (w & 3) .. +63 of the 256-row tile and K 64 (w >> 2) .. +63
-//               of each 256-K stage, so a token value is read from shared
-//               memory by 4 warps (not 16).  At the end of a unit the four
-//               K-group warps of a row group exchange partial sums through
-//               shared memory so that each owns a quarter of the outputs,
-//               summed over K groups in a fixed order (deterministic), and
-//               runs the epilogue for it.
+//   warps 0-15  compute: warp w owns 16 rows of the 256-row tile (gate/up:
+//               the gate and up rows of features 8w .. 8w+7) and all of each
+//               256-K stage, so it finishes its outputs alone: no partial
+//               sums change hands inside the CTA and the epilogue needs no
+//               barrier.
 //   warp 16     takes units from the queue; TMA of the 256 weight rows (two
 //               128-row boxes of codes, 128-byte swizzle, and of scales)
 //   warp 17     TMA of the unit's token rows (16-row boxes of the permuted f16
 //               activations or of h), after the dependency wait for down units
 //
 // K permutation.  A dot product may visit K in any order as long as both
-// operands use the same order.  Thread t of each quad supplies logical k in
-// {2t, 2t+1, 2t+8, 2t+9} of MMA step i (0..3) of its 64-K slice; they are
-// mapped to physical k = 16 t + 4 i + {0, 1, 2, 3}.  So a thread's 16 K of a
-// row are one 16-element NVFP4 scale block (one 8-byte load of codes, one
-// scale byte), and its token values are 16 consecutive K (two 16-byte loads).
+// operands use the same order.  For MMA step i (0..7) of a 128-K half stage,
+// thread t of each quad supplies logical k in {2t, 2t+1, 2t+8, 2t+9}; they
+// are mapped to physical k = 32 t + 4 i + {0, 1, 2, 3}.  So a thread's codes
+// for all eight steps are 32 consecutive K of its row (one 16-byte load, two
+// scale bytes), and its token values are 32 consecutive K of the token row
+// (four 16-byte loads per token tile).
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include "sm100.cuh"
@@ -60,10 +58,9 @@ constexpr int kDecWStageBytes = kDecCodes + kDecRows * 16; // + 256 rows x 16 B 
 constexpr int kDecBBoxBytes = kDecBN * 128;               // 64 K x 16 rows of f16
 constexpr int kDecBStageBytes = 4 * kDecBBoxBytes;        // 256 K
 constexpr int kDecStageBytes = kDecWStageBytes + kDecBStageBytes;
-constexpr int kDecRedBytes = 4 * 3 * 4 * 2 * 32 * 16;     // owner quarter x 3 sources x row groups x n-tiles x lanes
 constexpr int kDecSmemBytes =
-    1024 + kDecStages * kDecStageBytes + kDecRedBytes + (2 * kDecStages + 2 * kDecUnitRing + 2) * 8 + 64;
-constexpr int kDecPartialBytes = 4 * 4 * 2 * 32 * 16;     // one unit's split-K partial sums (row group x quarter x n-tile x lane)
+    1024 + kDecStages * kDecStageBytes + (2 * kDecStages + 2 * kDecUnitRing) * 8 + 128;
+constexpr int kDecPartialBytes = 16 * 2 * 32 * 16;        // one unit's split-K partial sums (warp x n-tile x lane)
 static_assert(kDecStageBytes % 1024 == 0, "stage alignment");
 static_assert(kDecSmemBytes <= 227 * 1024, "shared memory budget");
 
@@ -114,12 +111,17 @@ struct DecUnit {
   int tile;            // token tile (same tiling for both GEMMs)
 };
 
-__device__ __forceinline__ DecUnit decode_unit(const DecodeParams& p, int q, int n1) {
+// Queue position q is unit q of gate/up (q < n1) or unit q - n1 of down.
+__device__ __forceinline__ int4 unit_desc(const DecodeParams& p, int q, int n1) {
+  return q < n1 ? p.g[0].units[q] : p.g[1].units[q - n1];
+}
+
+// v: the unit's descriptor {expert | slot << 10, m-tile, first row, rows | split << 16}
+__device__ __forceinline__ DecUnit decode_unit(const DecodeParams& p, int q, int n1, const int4 v) {
   DecUnit d;
   d.gemm = q < n1 ? 0 : 1;
   d.u = d.gemm ? q - n1 : q;
   const FfnParams& g = p.g[d.gemm];
-  const int4 v = g.units[d.u];
   d.e = v.x & 1023; d.slot = v.x >> 10;
   d.mt = v.y; d.rb = v.z; d.nr = v.w & 0xFFFF;
   d.split = v.w >> 16;
@@ -130,82 +132,61 @@ __device__ __forceinline__ DecUnit decode_unit(const DecodeParams& p, int q, int
   return d;
 }
 
-// Stage-relative row of m-tile j (16 rows) of row group mg.  Gate/up stages
-// hold the 128 gate rows then the 128 up rows of the same features; row group
-// mg takes gate features 32 mg .. +31 (m-tiles 0, 1) and the up rows of the
-// same features (m-tiles 2, 3), so one thread ends up with both halves of
-// each SwiGLU.  Down stages: rows 64 mg + 16 j.
-__device__ __forceinline__ int dec_row_base(int gemm, int mg, int j) {
-  return gemm ? 64 * mg + 16 * j : (j < 2 ? 32 * mg + 16 * j : kDecFeat1 + 32 * mg + 16 * (j - 2));
+// Rows of the 256-row stage that warp w covers as the A rows g and g + 8 of
+// its m16 tiles.  Gate/up stages hold the 128 gate rows then the 128 up rows
+// of the same features; warp w takes features 8w .. 8w+7 -- their gate rows
+// as A rows g and their up rows as A rows g + 8 -- so each thread ends up
+// with both halves of its SwiGLUs.  Down stages: rows 16w .. 16w+15.
+__device__ __forceinline__ int dec_row_lo(int gemm, int w, int g) { return gemm ? 16 * w + g : 8 * w + g; }
+__device__ __forceinline__ int dec_row_hi(int gemm, int w, int g) {
+  return gemm ? 16 * w + 8 + g : kDecFeat1 + 8 * w + g;
 }
 
-// One 256-K stage for this warp: its 64 rows (4 m-tiles) x its 64 K x NT
-// token tiles of 8.
+// One 256-K stage for this warp: its 16 rows x 256 K x NT token tiles of 8.
 template <int NT>
-__device__ __forceinline__ void dec_stage(const uint8_t* st, const int (&rlo)[4], int kg, int g, int t,
-                                          float (&acc)[4][NT][4]) {
-  const uint8_t* bbox = st + kDecWStageBytes + kg * kDecBBoxBytes;
-  uint4 bt[NT][2];
+__device__ __forceinline__ void dec_stage(const uint8_t* st, int r_lo, int r_hi, int g, int t,
+                                          float (&acc)[NT][4]) {
+  const uint8_t* bst = st + kDecWStageBytes;
 #pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const int row = 8 * n + g;   // token row; its 16 K are 16-byte chunks 2t, 2t+1 (swizzled)
-    bt[n][0] = *reinterpret_cast<const uint4*>(bbox + row * 128 + (((2 * t) ^ (row & 7)) << 4));
-    bt[n][1] = *reinterpret_cast<const uint4*>(bbox + row * 128 + (((2 * t + 1) ^ (row & 7)) << 4));
-  }
-  const int cchunk = 2 * kg + (t >> 1), cbyte = 8 * (t & 1);
-  const uint8_t* sc = st + kDecCodes + 4 * kg + t;
+  for (int h = 0; h < 2; ++h) {   // 128-K halves: thread t covers K 128h + 32t .. +31
+    const uint8_t* bbox = bst + (2 * h + (t >> 1)) * kDecBBoxBytes;
+    const int chunk = 4 * h + t;   // 16-byte chunk of the 128-byte codes row: 32 codes
+    const uint4 clo = *reinterpret_cast<const uint4*>(st + r_lo * 128 + ((chunk ^ (r_lo & 7)) << 4));
+    const uint4 chi = *reinterpret_cast<const uint4*>(st + r_hi * 128 + ((chunk ^ (r_hi & 7)) << 4));
+    const uint32_t slo = *reinterpret_cast<const uint16_t*>(st + kDecCodes + r_lo * 16 + 8 * h + 2 * t);
+    const uint32_t shi = *reinterpret_cast<const uint16_t*>(st + kDecCodes + r_hi * 16 + 8 * h + 2 * t);
+    const uint32_t wlo[4] = {clo.x, clo.y, clo.z, clo.w};
+    const uint32_t whi[4] = {chi.x, chi.y, chi.z, chi.w};
+    // the thread's 32 K span two 16-K scale blocks: words 0, 1 and words 2, 3
+    const uint32_t sl2[2] = {e4m3_pair_to_f16x2(slo & 0xFFu), e4m3_pair_to_f16x2(slo >> 8)};
+    const uint32_t sh2[2] = {e4m3_pair_to_f16x2(shi & 0xFFu), e4m3_pair_to_f16x2(shi >> 8)};
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int rl = rlo[j], rh = rl + 8;
-    const uint2 clo = *reinterpret_cast<const uint2*>(st + rl * 128 + ((cchunk ^ (rl & 7)) << 4) + cbyte);
-    const uint2 chi = *reinterpret_cast<const uint2*>(st + rh * 128 + ((cchunk ^ (rh & 7)) << 4) + cbyte);
-    const uint32_t sl = e4m3_pair_to_f16x2(sc[rl * 16]);
-    const uint32_t sh = e4m3_pair_to_f16x2(sc[rh * 16]);
-    uint32_t ql[2][4], qh[2][4];
-    e2m1x8_to_f16x2(clo.x, ql[0]);
-    e2m1x8_to_f16x2(clo.y, ql[1]);
-    e2m1x8_to_f16x2(chi.x, qh[0]);
-    e2m1x8_to_f16x2(chi.y, qh[1]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {   // physical k 16t + 4i + {0,1} (a0/a1, b0) and + {2,3} (a2/a3, b1)
-      const int w = i >> 1, o = (i & 1) * 2;
-      const uint32_t a0 = hmul2_f16(ql[w][o], sl), a1 = hmul2_f16(qh[w][o], sh);
-      const uint32_t a2 = hmul2_f16(ql[w][o + 1], sl), a3 = hmul2_f16(qh[w][o + 1], sh);
+    for (int wd = 0; wd < 4; ++wd) {   // word wd: 8 K = two MMA steps
+      const int cb = (t & 1) * 4 + wd;   // the token values of those 8 K: 16-byte chunk of the box row
+      uint4 bv[NT];
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        const uint4& b = bt[n][i >> 1];
-        mma_f16_16816(acc[j][n], a0, a1, a2, a3, (i & 1) ? b.z : b.x, (i & 1) ? b.w : b.y);
+        const int row = 8 * n + g;
+        bv[n] = *reinterpret_cast<const uint4*>(bbox + row * 128 + ((cb ^ (row & 7)) << 4));
+      }
+      const uint32_t sl = sl2[wd >> 1], sh = sh2[wd >> 1];
+      uint32_t qlo[4], qhi[4];
+      e2m1x8_to_f16x2(wlo[wd], qlo);
+      e2m1x8_to_f16x2(whi[wd], qhi);
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {   // physical k 4p + {0,1} (a0/a1, b0) and + {2,3} (a2/a3, b1)
+        const uint32_t a0 = hmul2_f16(qlo[2 * p], sl), a1 = hmul2_f16(qhi[2 * p], sh);
+        const uint32_t a2 = hmul2_f16(qlo[2 * p + 1], sl), a3 = hmul2_f16(qhi[2 * p + 1], sh);
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+          mma_f16_16816(acc[n], a0, a1, a2, a3, p ? bv[n].z : bv[n].x, p ? bv[n].w : bv[n].y);
       }
     }
   }
 }
 
-// Output quarters.  After the main loop the four K-group warps of a row group
-// split the row group's outputs four ways: warp kg owns quarter kg, i.e.
-// m-tiles p = kg & 1 and p + 2, fragment half hh = kg >> 1 (rows g + 8 hh),
-// every token tile.  For gate/up that is gate and up of the same features (a
-// whole SwiGLU); for down, two 16-row m-tiles.  Per token tile a quarter is
-// one float4: {m-tile p: token 2t, 2t+1;  m-tile p+2: token 2t, 2t+1}.
-template <int NT>
-__device__ __forceinline__ float4 dec_quarter(const float (&acc)[4][NT][4], int qq, int n) {
-  const int p = qq & 1, hh = qq >> 1;
-  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int pp = 0; pp < 2; ++pp)
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2)
-      if (pp == p && h2 == hh)
-        v = make_float4(acc[pp][n][2 * h2], acc[pp][n][2 * h2 + 1], acc[pp + 2][n][2 * h2], acc[pp + 2][n][2 * h2 + 1]);
-  return v;
-}
-
-__device__ __forceinline__ void add4(float4& a, const float4& b) { a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w; }
-
-// Epilogue of warp (mg, kg) for its quarter, once `v` holds the CTA's sums.
-// With split-K across CTAs the quarter is first left as a partial sum; the
-// last split to arrive adds all splits in order and finishes.
-// Per-unit epilogue constants, loaded when the unit starts so that their
-// latency hides behind the main loop.
+// Per-unit epilogue constants, loaded by the weight producer while the unit
+// streams in, and handed over through the unit ring.
 struct DecConsts {
   float g0, g1;        // global scales: gate and up (gate/up unit) or down twice
   int any_scaled;      // gate/up: some token row was prescaled to fit f16
@@ -221,37 +202,41 @@ __device__ __forceinline__ DecConsts dec_consts(const DecodeParams& p, const Dec
   return c;
 }
 
+// Epilogue of warp w for its 16 rows.  With split-K across CTAs the warp
+// first leaves its partial sums; the last split to arrive adds all splits
+// in a fixed order and finishes.  Gate/up: publishes the finished h rows to
+// the down units' token loaders (release after the warp's stores; the
+// loader acquires the count and fences before its TMA reads).
 template <int NT>
-__device__ __forceinline__ void dec_epilogue(const DecodeParams& p, const DecUnit& d, const DecConsts& c, int mg,
-                                             int kg, int lane, float4 (&v)[NT]) {
+__device__ __forceinline__ void dec_epilogue(const DecodeParams& p, const DecUnit& d, const DecConsts& c, int w,
+                                             int lane, float (&acc)[NT][4]) {
   const FfnParams& G = p.g[d.gemm];
   const int g = lane >> 2, t = lane & 3;
   if (G.splits > 1) {
-    // leave the partial quarter; the last split to arrive (acquire) sums them
     float4* part = reinterpret_cast<float4*>(G.partials);
     constexpr int kPer = kDecPartialBytes / 16;
-    const int slot = ((mg * 4 + kg) * 2) * 32 + lane;
+    const int slot = (w * 2) * 32 + lane;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) part[size_t(d.u) * kPer + slot + n * 32] = v[n];
+    for (int n = 0; n < NT; ++n)
+      part[size_t(d.u) * kPer + slot + n * 32] = make_float4(acc[n][0], acc[n][1], acc[n][2], acc[n][3]);
     __syncwarp();
     int last = 0;
-    if (lane == 0)
-      last = atom_acq_rel_gpu_add(G.counters + (d.u / G.splits) * 16 + mg * 4 + kg, 1) == G.splits - 1;
+    if (lane == 0) last = atom_acq_rel_gpu_add(G.counters + (d.u / G.splits) * 16 + w, 1) == G.splits - 1;
     last = __shfl_sync(0xFFFFFFFFu, last, 0);
     if (!last) return;
     const int u0 = d.u - d.split;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp = 0; sp < G.splits; ++sp)   // fixed order: the same sums whoever arrives last
-        add4(s, __ldcg(part + size_t(u0 + sp) * kPer + slot + n * 32));
-      v[n] = s;
+      for (int sp = 0; sp < G.splits; ++sp) {   // fixed order: the same sums whoever arrives last
+        const float4 v = __ldcg(part + size_t(u0 + sp) * kPer + slot + n * 32);
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+      acc[n][0] = s.x; acc[n][1] = s.y; acc[n][2] = s.z; acc[n][3] = s.w;
     }
   }
-  const int pq = kg & 1, hh = kg >> 1;
   if (d.gemm == 0) {
-    const float gs = c.g0, gu = c.g1;
-    const int f = d.mt * kDecFeat1 + 32 * mg + 16 * pq + g + 8 * hh;
+    const int f = d.mt * kDecFeat1 + 8 * w + g;
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -259,18 +244,14 @@ __device__ __forceinline__ void dec_epilogue(const DecodeParams& p, const DecUni
         const int r = 8 * n + 2 * t + e;
         if (r < d.nr && f < G.M) {
           const float ts = c.any_scaled ? __ldg(G.tokscale + __ldg(G.perm_src + d.rb + r) / G.k_top) : 1.0f;
-          const float gv = e ? v[n].y : v[n].x, uv = e ? v[n].w : v[n].z;
-          store_out<2>(G.out, size_t(d.rb + r) * G.M + f, silu_mul(gs * ts * gv, gu * ts * uv));
+          store_out<2>(G.out, size_t(d.rb + r) * G.M + f, silu_mul(c.g0 * ts * acc[n][e], c.g1 * ts * acc[n][2 + e]));
         }
       }
-    // publish (release, after the warp's stores; the reader acquires the count
-    // and orders its TMA reads behind it with a proxy fence)
     fence_proxy_async_global();
     __syncwarp();
     if (lane == 0) red_release_gpu_add(p.tile_done + d.tile, 1);
   } else {
-    const float gd = c.g0;
-    const int f = d.mt * kDecRows + 64 * mg + 16 * pq + g + 8 * hh;
+    const int f = d.mt * kDecRows + 16 * w + g;
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -278,52 +259,39 @@ __device__ __forceinline__ void dec_epilogue(const DecodeParams& p, const DecUni
         const int r = 8 * n + 2 * t + e;
         if (r < d.nr) {
           float* o = static_cast<float*>(G.out) + size_t(d.rb + r) * G.M;
-          if (f < G.M) o[f] = gd * (e ? v[n].y : v[n].x);
-          if (f + 32 < G.M) o[f + 32] = gd * (e ? v[n].w : v[n].z);
+          if (f < G.M) o[f] = c.g0 * acc[n][e];
+          if (f + 8 < G.M) o[f + 8] = c.g0 * acc[n][2 + e];
         }
       }
   }
 }
 
-// Barrier tags of the unit ring and of the K-group hand-off.
+// Barrier tag of the unit ring.
 constexpr int kTagUnit = 10;
-constexpr int kTagRed = 11;
 
-struct DecBars {
-  uint64_t* full;      // [kDecStages]  weights + tokens of a stage landed (2 arrivals + bytes)
-  uint64_t* empty;     // [kDecStages]  the 16 compute warps are done with a stage
-  uint64_t* redfull;   // all 16 compute warps stored their partial quarters (512 threads)
-  uint64_t* redfree;   // all 16 read theirs (512 threads)
-};
-
-// The main loop, K-group hand-off and epilogue of one unit for compute warp
-// (mg, kg).  `si` counts stages consumed by this CTA, `j` units.  The unit's
-// ring slot is released after the main loop, so a CTA takes a new unit from
-// the queue only when it has finished computing the one before the current
-// one: no CTA hoards small units while others idle.  Returns false if a wait
-// gave up (the kernel then winds down).
+// Main loop and epilogue of one unit for compute warp w.  `si` counts stages
+// consumed by this CTA.  The unit's ring slot is released after the main
+// loop, so a CTA takes a new unit from the queue only when it has finished
+// computing the one before the current one: no CTA hoards small units while
+// others idle.  Returns false if a wait gave up (the kernel then winds down).
 template <int NT>
-__device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem, float4* red, const DecBars& b,
-                         const Abort& ab, uint64_t* unit_free, const int4* unit_ent, uint32_t& si, int j, int q,
-                         int mg, int kg, int lane) {
+__device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem, uint64_t* full, uint64_t* empty,
+                         const Abort& ab, uint64_t* unit_free, const int4* unit_ent, uint32_t& si, int q, int w,
+                         int lane) {
   const int g = lane >> 2, t = lane & 3;
-  int rlo[4];
+  const int r_lo = dec_row_lo(d.gemm, w, g), r_hi = dec_row_hi(d.gemm, w, g);
+  float acc[NT][4];
 #pragma unroll
-  for (int jj = 0; jj < 4; ++jj) rlo[jj] = dec_row_base(d.gemm, mg, jj) + g;
-  float acc[4][NT][4];
+  for (int n = 0; n < NT; ++n)
 #pragma unroll
-  for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[jj][n][i] = 0.0f;
+    for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
 
   for (int ws = d.ws0; ws < d.ws1; ++ws, ++si) {
     const int s = si % kDecStages;
-    if (!__all_sync(0xFFFFFFFFu, ab.wait(&b.full[s], (si / kDecStages) & 1, kTagWFull, si, q))) return false;
-    dec_stage<NT>(smem + s * kDecStageBytes, rlo, kg, g, t, acc);
+    if (!__all_sync(0xFFFFFFFFu, ab.wait(&full[s], (si / kDecStages) & 1, kTagWFull, si, q))) return false;
+    dec_stage<NT>(smem + s * kDecStageBytes, r_lo, r_hi, g, t, acc);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&b.empty[s]);
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
   DecConsts c;   // written by the weight producer before the last stage (acquired above)
   {
@@ -332,29 +300,7 @@ __device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem,
   }
   __syncwarp();
   if (lane == 0) mbar_arrive(unit_free);   // the queue may hand this CTA its next-but-one unit
-
-  // hand the other three quarters to their owners; red[owner][source][mg][n][lane]
-  auto slot = [&](int owner, int src, int n) {
-    return red + ((((owner * 3 + (src < owner ? src : src - 1)) * 4 + mg) * 2 + n) * 32 + lane);
-  };
-  if (j > 0 && !__all_sync(0xFFFFFFFFu, ab.wait(b.redfree, (j - 1) & 1, kTagRed, j, q))) return false;
-#pragma unroll
-  for (int qq = 0; qq < 4; ++qq)
-    if (qq != kg)
-#pragma unroll
-      for (int n = 0; n < NT; ++n) *slot(qq, kg, n) = dec_quarter<NT>(acc, qq, n);
-  mbar_arrive(b.redfull);
-  if (!__all_sync(0xFFFFFFFFu, ab.wait(b.redfull, j & 1, kTagRed, j, q))) return false;
-  float4 v[NT];
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    v[n] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int src = 0; src < 4; ++src)   // K groups in order: deterministic sums
-      add4(v[n], src == kg ? dec_quarter<NT>(acc, kg, n) : *slot(kg, src, n));
-  }
-  mbar_arrive(b.redfree);
-  dec_epilogue<NT>(p, d, c, mg, kg, lane, v);
+  dec_epilogue<NT>(p, d, c, w, lane, acc);
   return true;
 }
 
@@ -399,23 +345,20 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
                   const __grid_constant__ CUtensorMap tm_h) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float4* red = reinterpret_cast<float4*>(smem + kDecStages * kDecStageBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecStages * kDecStageBytes + kDecRedBytes);
-  DecBars b{bars, bars + kDecStages, bars + 2 * kDecStages + 2 * kDecUnitRing,
-            bars + 2 * kDecStages + 2 * kDecUnitRing + 1};
-  uint64_t* ufull = bars + 2 * kDecStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecStages * kDecStageBytes);
+  uint64_t* empty = full + kDecStages;
+  uint64_t* ufull = empty + kDecStages;
   uint64_t* uempty = ufull + kDecUnitRing;
   // ring entries: {queue position, then (before the unit's last stage lands)
   // the epilogue constants: global scale bits x2, any token prescaled}
-  int4* uent = reinterpret_cast<int4*>(bars + 2 * kDecStages + 2 * kDecUnitRing + 2);
-  int* abort_flag = reinterpret_cast<int*>(uent + kDecUnitRing);
+  int4* uent = reinterpret_cast<int4*>(uempty + kDecUnitRing);
+  int4* udesc = uent + kDecUnitRing;   // [kDecUnitRing] the unit's descriptor, read once by the producer
+  int* abort_flag = reinterpret_cast<int*>(udesc + kDecUnitRing);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kDecStages; ++i) { mbar_init(&b.full[i], 2); mbar_init(&b.empty[i], 16); }
+    for (int i = 0; i < kDecStages; ++i) { mbar_init(&full[i], 2); mbar_init(&empty[i], 16); }
     for (int i = 0; i < kDecUnitRing; ++i) { mbar_init(&ufull[i], 1); mbar_init(&uempty[i], 17); }
-    mbar_init(b.redfull, 512);
-    mbar_init(b.redfree, 512);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -439,10 +382,12 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
         if (!(ok = ab.wait(&uempty[us], ((j / kDecUnitRing) & 1) ^ 1, kTagUnit, j, -3))) break;
         int q = atomicAdd(p.queue, 1);
         if (q >= ntot) q = -1;
+        const int4 raw = q >= 0 ? unit_desc(p, q, n1) : make_int4(0, 0, 0, 0);
+        udesc[us] = raw;
         uent[us].x = q;
         mbar_arrive(&ufull[us]);
         if (q < 0) break;
-        const DecUnit d = decode_unit(p, q, n1);
+        const DecUnit d = decode_unit(p, q, n1, raw);
         const DecConsts c = dec_consts(p, d);
         const int slot = d.slot;
         const CUtensorMap* c0 = d.gemm ? &tm_c2 : &tm_c0;
@@ -453,18 +398,18 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
         const int y1 = d.gemm ? y0 + 128 : y0;
         for (int ws = d.ws0; ws < d.ws1; ++ws, ++si) {
           const int s = si % kDecStages;
-          if (!(ok = ab.wait(&b.empty[s], ((si / kDecStages) & 1) ^ 1, kTagWEmpty, si, q))) break;
+          if (!(ok = ab.wait(&empty[s], ((si / kDecStages) & 1) ^ 1, kTagWEmpty, si, q))) break;
           if (ws == d.ws1 - 1)   // published by this stage's arrival (release) to the compute warps
             uent[us] = make_int4(q, __float_as_int(c.g0), __float_as_int(c.g1), c.any_scaled);
-          mbar_arrive_expect_tx(&b.full[s], kDecWStageBytes);
+          mbar_arrive_expect_tx(&full[s], kDecWStageBytes);
           uint8_t* st = smem + s * kDecStageBytes;
-          tma_load_3d(st, c0, &b.full[s], ws * 128, y0, slot);
-          tma_load_3d(st + 128 * 128, c1, &b.full[s], ws * 128, y1, slot);
-          tma_load_3d(st + kDecCodes, s0, &b.full[s], ws * 16, y0, slot);
-          tma_load_3d(st + kDecCodes + 128 * 16, s1, &b.full[s], ws * 16, y1, slot);
+          tma_load_3d(st, c0, &full[s], ws * 128, y0, slot);
+          tma_load_3d(st + 128 * 128, c1, &full[s], ws * 128, y1, slot);
+          tma_load_3d(st + kDecCodes, s0, &full[s], ws * 16, y0, slot);
+          tma_load_3d(st + kDecCodes + 128 * 16, s1, &full[s], ws * 16, y1, slot);
         }
       }
-      dec_drain(b.full, si);
+      dec_drain(full, si);
     }
   } else if (warp == 17) {
     // ------------------------------------------------- token TMA ---
@@ -476,7 +421,7 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
         if (!(ok = ab.wait(&ufull[us], (j / kDecUnitRing) & 1, kTagUnit, j, -1))) break;
         const int q = uent[us].x;
         if (q < 0) { mbar_arrive(&uempty[us]); break; }
-        const DecUnit d = decode_unit(p, q, n1);
+        const DecUnit d = decode_unit(p, q, n1, udesc[us]);
         if (d.gemm == 1) {
           if (!(ok = dec_wait_h(p, d, ab, q))) break;
           fence_proxy_async_global();   // the h rows were written by generic stores
@@ -484,20 +429,19 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
         const CUtensorMap* act = d.gemm ? &tm_h : &tm_x;
         for (int ws = d.ws0; ws < d.ws1; ++ws, ++si) {
           const int s = si % kDecStages;
-          if (!(ok = ab.wait(&b.empty[s], ((si / kDecStages) & 1) ^ 1, kTagBEmpty, si, q))) break;
-          mbar_arrive_expect_tx(&b.full[s], kDecBStageBytes);
+          if (!(ok = ab.wait(&empty[s], ((si / kDecStages) & 1) ^ 1, kTagBEmpty, si, q))) break;
+          mbar_arrive_expect_tx(&full[s], kDecBStageBytes);
           uint8_t* bst = smem + s * kDecStageBytes + kDecWStageBytes;
 #pragma unroll
           for (int bx = 0; bx < 4; ++bx)
-            tma_load_2d(bst + bx * kDecBBoxBytes, act, &b.full[s], ws * kDecStageK + bx * 64, d.rb);
+            tma_load_2d(bst + bx * kDecBBoxBytes, act, &full[s], ws * kDecStageK + bx * 64, d.rb);
         }
         mbar_arrive(&uempty[us]);
       }
-      dec_drain(b.full, si);
+      dec_drain(full, si);
     }
   } else {
     // --------------------------------------------------- compute ---
-    const int mg = warp & 3, kg = warp >> 2;
     uint32_t si = 0;
     for (int j = 0;; ++j) {
       const int us = j % kDecUnitRing;
@@ -508,9 +452,9 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
         if (lane == 0) mbar_arrive(&uempty[us]);
         break;
       }
-      const DecUnit d = decode_unit(p, q, n1);
-      const bool ok = d.nr > 8 ? dec_unit<2>(p, d, smem, red, b, ab, &uempty[us], &uent[us], si, j, q, mg, kg, lane)
-                               : dec_unit<1>(p, d, smem, red, b, ab, &uempty[us], &uent[us], si, j, q, mg, kg, lane);
+      const DecUnit d = decode_unit(p, q, n1, udesc[us]);
+      const bool ok = d.nr > 8 ? dec_unit<2>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], si, q, warp, lane)
+                               : dec_unit<1>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], si, q, warp, lane);
       if (!ok) break;
     }
   }
