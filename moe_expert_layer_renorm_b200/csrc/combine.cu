@@ -13,6 +13,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
                                                       const int32_t* __restrict__ pair_to_row,
                                                       const float* __restrict__ w, int T, int k, int H,
                                                       int P, float4* __restrict__ y) {
+  pdl_enter();
   const int vec_per_row = H / 4;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)T * vec_per_row) return;
@@ -37,9 +38,8 @@ static cudaError_t launch_combine(const void* out_perm, const int32_t* pair_to_r
   const int threads = 256;
   const long long blocks = (n + threads - 1) / threads;
   ProfileScope prof(FT_KERNEL_COMBINE, s);
-  combine_kernel<<<dim3(unsigned(blocks)), threads, 0, s>>>(static_cast<const float4*>(out_perm), pair_to_row,
-                                                            w, T, k, H, T * k, static_cast<float4*>(y));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(unsigned(blocks)), dim3(threads), 0, s,
+                    static_cast<const float4*>(out_perm), pair_to_row, w, T, k, H, T * k, static_cast<float4*>(y));
 }
 
 }  // namespace ftmoe

@@ -343,6 +343,7 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
                   const __grid_constant__ CUtensorMap tm_s1, const __grid_constant__ CUtensorMap tm_c2,
                   const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_x,
                   const __grid_constant__ CUtensorMap tm_h) {
+  pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecStages * kDecStageBytes);
@@ -471,9 +472,8 @@ static cudaError_t launch_decode(const DecodeParams& p, int grid, const CUtensor
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  ffn_decode_kernel<<<grid, kDecThreads, kDecSmemBytes, s>>>(p, tmc[0], tms[0], tmc[1], tms[1], tmc[2], tms[2],
-                                                             tm_x, tm_h);
-  return cudaGetLastError();
+  return launch_pdl(ffn_decode_kernel, dim3(grid), dim3(kDecThreads), kDecSmemBytes, s, p, tmc[0], tms[0], tmc[1],
+                    tms[1], tmc[2], tms[2], tm_x, tm_h);
 }
 
 }  // namespace ftmoe

@@ -154,7 +154,10 @@ struct Abort {
   }
 };
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u = g * u / (1 + e^-g).  The hardware exponential and a fast
+// divide: a few ulps of fp32, far inside the layer's tolerance; as g -> -inf
+// the divisor overflows to inf and the result goes to 0, its limit.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g * u, 1.0f + __expf(-g)); }
 
 // GEMM1 stores h in f16 (it is the next MMA's operand; a value beyond the f16
 // range saturates and records FT_DEV_F16_RANGE); GEMM2 stores the expert
@@ -184,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0,
                 const __grid_constant__ CUtensorMap tm_scales0, const __grid_constant__ CUtensorMap tm_codes1,
                 const __grid_constant__ CUtensorMap tm_scales1, const __grid_constant__ CUtensorMap tm_act) {
+  pdl_enter();
   using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -394,6 +398,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
       float gsc[NMAT];
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) gsc[m] = __ldg(reinterpret_cast<const float*>(sbase + p.global_off[m]));
+      const int any_scaled = NMAT == 2 && p.perm_src != nullptr ? *p.any_scaled : 0;
       if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&d_full[ds], (di / DB) & 1, kTagDFull, di, u)))) break;
       tc_fence_after();
       const int n_eff = (nr + 15) & ~15;
@@ -414,7 +419,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
           } else if (feat < p.M) {
             float r;
             if (NMAT == 2) {
-              const float ts = token_factor(p, rb + n);
+              const float ts = any_scaled ? token_factor(p, rb + n) : 1.0f;
               r = silu_mul(gsc[0] * ts * __uint_as_float(v[0][i]), gsc[NMAT - 1] * ts * __uint_as_float(v[NMAT - 1][i]));
             } else {
               r = gsc[0] * __uint_as_float(v[0][i]);
@@ -449,7 +454,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
             if (feat < p.M) {
               float r;
               if (NMAT == 2) {
-                const float ts = token_factor(p, rb + n);
+                const float ts = any_scaled ? token_factor(p, rb + n) : 1.0f;
                 r = silu_mul(gsc[0] * ts * acc[0], gsc[NMAT - 1] * ts * acc[NMAT - 1]);
               } else {
                 r = gsc[0] * acc[0];
@@ -484,6 +489,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
 __global__ void __launch_bounds__(256) prep_x_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_src,
                                                      int P, int k_top, int H, uint4* __restrict__ x_perm,
                                                      float* __restrict__ tokscale, int* __restrict__ any_scaled) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int r = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (r >= P) return;
@@ -539,6 +545,7 @@ __global__ void __launch_bounds__(1024) ffn_schedule_kernel(
     int bn1, int mt1, int s1, int bn2, int mt2, int s2, int4* __restrict__ units1, int4* __restrict__ units2,
     int* __restrict__ counts, int* __restrict__ counters1, int ncnt1, int* __restrict__ counters2, int ncnt2,
     int* __restrict__ tile_done, int ndone) {
+  pdl_enter();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
   int n = 0, rb = 0, slot = 0;

@@ -192,8 +192,7 @@ static cudaError_t launch_gemm(const FfnParams& p, int grid, const CUtensorMap& 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, kThreads, Cfg::kSmemBytes, s>>>(p, c0, s0, c1, s1, act);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), Cfg::kSmemBytes, s, p, c0, s0, c1, s1, act);
 }
 
 static int device_sm_count() {
@@ -225,22 +224,20 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   __half* h = reinterpret_cast<__half*>(w + pl.off_h);
   __half* x16 = reinterpret_cast<__half*>(w + pl.off_x16);
   float* tokscale = reinterpret_cast<float*>(w + pl.off_tokscale);
+  cudaError_t err;
   {
-  ProfileScope prof(FT_KERNEL_SCHEDULE, s);
-  ffn_schedule_kernel<<<1, 1024, 0, s>>>(offsets, slot_table, E, L.num_slots, pl.g1.bn, pl.mt1, pl.g1.splits,
-                                         pl.g2.bn, pl.mt2, pl.g2.splits, units1, units2, counts, cnt1,
-                                         int(pl.max_tiles1 * pl.mt1 * pl.cnt_per), cnt2,
-                                         int(pl.max_tiles2 * pl.mt2 * pl.cnt_per),
-                                         reinterpret_cast<int*>(w + pl.off_done), pl.decode ? int(pl.max_tiles1) : 0);
+    ProfileScope prof(FT_KERNEL_SCHEDULE, s);
+    err = launch_pdl(ffn_schedule_kernel, dim3(1), dim3(1024), 0, s, offsets, slot_table, E, L.num_slots, pl.g1.bn,
+                     pl.mt1, pl.g1.splits, pl.g2.bn, pl.mt2, pl.g2.splits, units1, units2, counts, cnt1,
+                     int(pl.max_tiles1 * pl.mt1 * pl.cnt_per), cnt2, int(pl.max_tiles2 * pl.mt2 * pl.cnt_per),
+                     reinterpret_cast<int*>(w + pl.off_done), pl.decode ? int(pl.max_tiles1) : 0);
   }
-  cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   {
     ProfileScope prof(FT_KERNEL_PREP, s);
-    prep_x_kernel<<<(T * k + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(x), perm_src, T * k, k, H,
-                                                  reinterpret_cast<uint4*>(x16), tokscale, counts + 2);
+    err = launch_pdl(prep_x_kernel, dim3((T * k + 7) / 8), dim3(256), 0, s, static_cast<const uint4*>(x), perm_src,
+                     T * k, k, H, reinterpret_cast<uint4*>(x16), tokscale, counts + 2);
   }
-  err = cudaGetLastError();
   if (err != cudaSuccess) return err;
 
   CUtensorMap tm_x, tm_h;

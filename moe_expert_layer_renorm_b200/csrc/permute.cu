@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
                                                              int32_t* __restrict__ offsets,
                                                              int32_t* __restrict__ perm_src,
                                                              int32_t* __restrict__ pair_to_row) {
+  pdl_enter();
   __shared__ int cnt[kMaxExperts];
   __shared__ int warp_sums[32];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
 
 __global__ void __launch_bounds__(256) permute_hist_kernel(const int32_t* __restrict__ ids, int P, int E,
                                                            int32_t* __restrict__ counts) {
+  pdl_enter();
   __shared__ int cnt[kMaxExperts];
   const int c = blockIdx.x;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -111,6 +113,7 @@ __global__ void __launch_bounds__(256) permute_hist_kernel(const int32_t* __rest
 
 __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ counts, int nchunks, int E,
                                                             int32_t* __restrict__ offsets) {
+  pdl_enter();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
   int total = 0;
@@ -133,6 +136,7 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __r
                                                               const int32_t* __restrict__ bases,
                                                               int32_t* __restrict__ perm_src,
                                                               int32_t* __restrict__ pair_to_row) {
+  pdl_enter();
   __shared__ int cursor[kMaxExperts];
   const int c = blockIdx.x;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] = bases[size_t(c) * E + e];
@@ -155,23 +159,23 @@ static cudaError_t launch_permute(const int32_t* ids, int T, int k, int E, int32
   const int nchunks = (P + kPermChunk - 1) / kPermChunk;
   if (nchunks <= 1) {
     ProfileScope prof(FT_KERNEL_PERMUTE, s);
-    permute_small_kernel<<<1, 1024, 0, s>>>(ids, P, E, offsets, perm_src, pair_to_row);
-    return cudaGetLastError();
+    return launch_pdl(permute_small_kernel, dim3(1), dim3(1024), 0, s, ids, P, E, offsets, perm_src, pair_to_row);
   }
   int32_t* counts = static_cast<int32_t*>(ws);
+  cudaError_t e;
   {
     ProfileScope prof(FT_KERNEL_PERMUTE, s);
-    permute_hist_kernel<<<nchunks, 256, 0, s>>>(ids, P, E, counts);
+    e = launch_pdl(permute_hist_kernel, dim3(nchunks), dim3(256), 0, s, ids, P, E, counts);
   }
+  if (e != cudaSuccess) return e;
   {
     ProfileScope prof(FT_KERNEL_PERMUTE, s);
-    permute_scan_kernel<<<1, 1024, 0, s>>>(counts, nchunks, E, offsets);
+    e = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, counts, nchunks, E, offsets);
   }
-  {
-    ProfileScope prof(FT_KERNEL_PERMUTE, s);
-    permute_scatter_kernel<<<nchunks, 256, 0, s>>>(ids, P, E, counts, perm_src, pair_to_row);
-  }
-  return cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ProfileScope prof(FT_KERNEL_PERMUTE, s);
+  return launch_pdl(permute_scatter_kernel, dim3(nchunks), dim3(256), 0, s, ids, P, E,
+                    static_cast<const int32_t*>(counts), perm_src, pair_to_row);
 }
 
 }  // namespace ftmoe

@@ -16,6 +16,7 @@ template <int NPL>  // logits per lane = ceil(E / 32)
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                      int mode, int32_t* __restrict__ ids,
                                                      float* __restrict__ wts) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (t >= T) return;
@@ -90,13 +91,9 @@ static cudaError_t launch_route(const float* logits, int T, int E, int k, int mo
   const dim3 grid((T + warps - 1) / warps), block(32 * warps);
   const int npl = (E + 31) / 32;
   ProfileScope prof(FT_KERNEL_ROUTE, s);
-  if (npl <= 1) route_kernel<1><<<grid, block, 0, s>>>(logits, T, E, k, mode, ids, w);
-  else if (npl <= 2) route_kernel<2><<<grid, block, 0, s>>>(logits, T, E, k, mode, ids, w);
-  else if (npl <= 4) route_kernel<4><<<grid, block, 0, s>>>(logits, T, E, k, mode, ids, w);
-  else if (npl <= 8) route_kernel<8><<<grid, block, 0, s>>>(logits, T, E, k, mode, ids, w);
-  else if (npl <= 16) route_kernel<16><<<grid, block, 0, s>>>(logits, T, E, k, mode, ids, w);
-  else route_kernel<32><<<grid, block, 0, s>>>(logits, T, E, k, mode, ids, w);
-  return cudaGetLastError();
+  auto kern = npl <= 1 ? route_kernel<1> : npl <= 2 ? route_kernel<2> : npl <= 4 ? route_kernel<4>
+             : npl <= 8 ? route_kernel<8> : npl <= 16 ? route_kernel<16> : route_kernel<32>;
+  return launch_pdl(kern, grid, block, 0, s, logits, T, E, k, mode, ids, w);
 }
 
 }  // namespace ftmoe

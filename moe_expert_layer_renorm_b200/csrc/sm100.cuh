@@ -6,6 +6,7 @@
 // records an error code in the library's device status word and returns
 // false, so a kernel never spins forever.
 #pragma once
+#include <utility>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -240,6 +241,35 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 // Named barrier for a subset of warps.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Programmatic dependent launch.  Every hot-path kernel starts with this:
+// wait until the grids it depends on have completed and their memory is
+// visible (a no-op when it was launched without such a dependency), then let
+// the next grid in the stream begin launching, so that its set-up overlaps
+// this grid's work instead of following it.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch with the programmatic-stream-serialisation attribute: the kernel
+// may start before the previous kernel in the stream ends, and waits for it
+// in pdl_enter().  Captured into CUDA graphs as a programmatic edge.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace ftmoe
