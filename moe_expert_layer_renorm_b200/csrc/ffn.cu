@@ -547,6 +547,8 @@ __global__ void __launch_bounds__(1024) ffn_schedule_kernel(
     int* __restrict__ tile_done, int ndone) {
   pdl_enter();
   __shared__ int warp_sums[32];
+  __shared__ int start1[kMaxExperts + 1], start2[kMaxExperts + 1];   // first tile of each expert
+  __shared__ int s_rb[kMaxExperts], s_n[kMaxExperts], s_slot[kMaxExperts];
   const int e = threadIdx.x;
   int n = 0, rb = 0, slot = 0;
   if (e < E) {
@@ -557,23 +559,38 @@ __global__ void __launch_bounds__(1024) ffn_schedule_kernel(
       if (slot < 0) { set_device_status(FT_DEV_NOT_RESIDENT); n = 0; }
       else if (slot >= num_slots) { set_device_status(FT_DEV_BAD_INDEX); n = 0; }
     }
+    s_rb[e] = rb;
+    s_n[e] = n;
+    s_slot[e] = slot;
   }
   const int t1 = (n + bn1 - 1) / bn1, t2 = (n + bn2 - 1) / bn2;
   const int ex1 = block_exclusive_scan(t1, warp_sums);
   const int ex2 = block_exclusive_scan(t2, warp_sums);
-  for (int t = 0; t < t1; ++t)
-    for (int m = 0; m < mt1; ++m)
-      for (int s = 0; s < s1; ++s)
-        units1[((ex1 + t) * mt1 + m) * s1 + s] =
-            make_int4(e | (slot << 10), m, rb + t * bn1, min(bn1, n - t * bn1) | (s << 16));
-  for (int t = 0; t < t2; ++t)
-    for (int m = 0; m < mt2; ++m)
-      for (int s = 0; s < s2; ++s)
-        units2[((ex2 + t) * mt2 + m) * s2 + s] =
-            make_int4(e | (slot << 10), m, rb + t * bn2, min(bn2, n - t * bn2) | (s << 16));
-  if (e == blockDim.x - 1) {
-    counts[0] = (ex1 + t1) * mt1 * s1;
-    counts[1] = (ex2 + t2) * mt2 * s2;
+  if (e < E) { start1[e] = ex1; start2[e] = ex2; }
+  if (e == E - 1) { start1[E] = ex1 + t1; start2[E] = ex2 + t2; }
+  __syncthreads();
+  // every thread writes units of every expert: u -> (tile, m-tile, split),
+  // the tile's expert by binary search over the experts' first tiles
+  auto fill = [&](const int* start, int bn, int mt, int sp, int4* units) {
+    const int total = start[E] * mt * sp;
+    for (int u = threadIdx.x; u < total; u += blockDim.x) {
+      const int tile = u / (mt * sp), rem = u - tile * (mt * sp);
+      int lo = 0, hi = E;                 // last expert whose first tile is <= tile
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (start[mid] <= tile) lo = mid; else hi = mid;
+      }
+      const int t = tile - start[lo];
+      units[u] = make_int4(lo | (s_slot[lo] << 10), rem / sp, s_rb[lo] + t * bn,
+                           min(bn, s_n[lo] - t * bn) | ((rem % sp) << 16));
+    }
+    return total;
+  };
+  const int total1 = fill(start1, bn1, mt1, s1, units1);
+  const int total2 = fill(start2, bn2, mt2, s2, units2);
+  if (threadIdx.x == 0) {
+    counts[0] = total1;
+    counts[1] = total2;
   }
   if (threadIdx.x == 0) { counts[2] = 0; counts[3] = 0; }   // any token prescaled; unit queue
   for (int i = threadIdx.x; i < ncnt1; i += blockDim.x) counters1[i] = 0;
