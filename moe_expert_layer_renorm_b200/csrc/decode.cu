@@ -22,7 +22,7 @@
 // published; every unit it waits on was taken earlier by a running CTA, so
 // the wait always ends.  The down unit's weights stream in meanwhile.
 //
-// CTA (18 warps):
+// CTA (19 warps):
 //   warps 0-15  compute: warp w owns 16 rows of the 256-row tile (gate/up:
 //               the gate and up rows of features 8w .. 8w+7) and all of each
 //               256-K stage, so it finishes its outputs alone: no partial
@@ -32,6 +32,8 @@
 //               128-row boxes of codes, 128-byte swizzle, and of scales)
 //   warp 17     TMA of the unit's token rows (16-row boxes of the permuted f16
 //               activations or of h), after the dependency wait for down units
+//   warp 18     publishes each gate/up unit's finished h rows to other CTAs
+//               with one release, so compute warps never wait on a fence
 //
 // K permutation.  A dot product may visit K in any order as long as both
 // operands use the same order.  For MMA step i (0..7) of a 128-K half stage,
@@ -46,7 +48,7 @@
 
 namespace ftmoe {
 
-constexpr int kDecThreads = 18 * 32;
+constexpr int kDecThreads = 19 * 32;
 constexpr int kDecRows = 256;      // weight rows per CTA tile (down); gate/up: 128 features x 2
 constexpr int kDecFeat1 = 128;     // gate/up features per tile
 constexpr int kDecBN = 16;         // token rows per unit
@@ -59,7 +61,7 @@ constexpr int kDecBBoxBytes = kDecBN * 128;               // 64 K x 16 rows of f
 constexpr int kDecBStageBytes = 4 * kDecBBoxBytes;        // 256 K
 constexpr int kDecStageBytes = kDecWStageBytes + kDecBStageBytes;
 constexpr int kDecSmemBytes =
-    1024 + kDecStages * kDecStageBytes + (2 * kDecStages + 2 * kDecUnitRing) * 8 + 128;
+    1024 + kDecStages * kDecStageBytes + (2 * kDecStages + 2 * kDecUnitRing + 2) * 8 + 128;
 constexpr int kDecPartialBytes = 16 * 2 * 32 * 16;        // one unit's split-K partial sums (warp x n-tile x lane)
 static_assert(kDecStageBytes % 1024 == 0, "stage alignment");
 static_assert(kDecSmemBytes <= 227 * 1024, "shared memory budget");
@@ -204,11 +206,10 @@ __device__ __forceinline__ DecConsts dec_consts(const DecodeParams& p, const Dec
 
 // Epilogue of warp w for its 16 rows.  With split-K across CTAs the warp
 // first leaves its partial sums; the last split to arrive adds all splits
-// in a fixed order and finishes.  Gate/up: publishes the finished h rows to
-// the down units' token loaders (release after the warp's stores; the
-// loader acquires the count and fences before its TMA reads).
+// in a fixed order and finishes.  Returns true if this warp stored the
+// outputs.
 template <int NT>
-__device__ __forceinline__ void dec_epilogue(const DecodeParams& p, const DecUnit& d, const DecConsts& c, int w,
+__device__ __forceinline__ bool dec_epilogue(const DecodeParams& p, const DecUnit& d, const DecConsts& c, int w,
                                              int lane, float (&acc)[NT][4]) {
   const FfnParams& G = p.g[d.gemm];
   const int g = lane >> 2, t = lane & 3;
@@ -223,7 +224,7 @@ __device__ __forceinline__ void dec_epilogue(const DecodeParams& p, const DecUni
     int last = 0;
     if (lane == 0) last = atom_acq_rel_gpu_add(G.counters + (d.u / G.splits) * 16 + w, 1) == G.splits - 1;
     last = __shfl_sync(0xFFFFFFFFu, last, 0);
-    if (!last) return;
+    if (!last) return false;
     const int u0 = d.u - d.split;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
@@ -247,9 +248,6 @@ __device__ __forceinline__ void dec_epilogue(const DecodeParams& p, const DecUni
           store_out<2>(G.out, size_t(d.rb + r) * G.M + f, silu_mul(c.g0 * ts * acc[n][e], c.g1 * ts * acc[n][2 + e]));
         }
       }
-    fence_proxy_async_global();
-    __syncwarp();
-    if (lane == 0) red_release_gpu_add(p.tile_done + d.tile, 1);
   } else {
     const int f = d.mt * kDecRows + 16 * w + g;
 #pragma unroll
@@ -264,6 +262,7 @@ __device__ __forceinline__ void dec_epilogue(const DecodeParams& p, const DecUni
         }
       }
   }
+  return true;
 }
 
 // Barrier tag of the unit ring.
@@ -276,8 +275,8 @@ constexpr int kTagUnit = 10;
 // others idle.  Returns false if a wait gave up (the kernel then winds down).
 template <int NT>
 __device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem, uint64_t* full, uint64_t* empty,
-                         const Abort& ab, uint64_t* unit_free, const int4* unit_ent, uint32_t& si, int q, int w,
-                         int lane) {
+                         const Abort& ab, uint64_t* unit_free, const int4* unit_ent, uint64_t* hpub, int* hcount,
+                         int gu, uint32_t& si, int q, int w, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int r_lo = dec_row_lo(d.gemm, w, g), r_hi = dec_row_hi(d.gemm, w, g);
   float acc[NT][4];
@@ -300,7 +299,12 @@ __device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem,
   }
   __syncwarp();
   if (lane == 0) mbar_arrive(unit_free);   // the queue may hand this CTA its next-but-one unit
-  dec_epilogue<NT>(p, d, c, w, lane, acc);
+  const bool fin = dec_epilogue<NT>(p, d, c, w, lane, acc);
+  if (d.gemm == 0) {   // gate/up: hand the h rows to the publisher
+    __syncwarp();
+    if (fin && lane == 0) atomicAdd(&hcount[gu & 1], 1);
+    mbar_arrive(&hpub[gu & 1]);   // after this thread's stores (release)
+  }
   return true;
 }
 
@@ -350,16 +354,19 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
   uint64_t* empty = full + kDecStages;
   uint64_t* ufull = empty + kDecStages;
   uint64_t* uempty = ufull + kDecUnitRing;
+  uint64_t* hpub = uempty + kDecUnitRing;   // [2] by gate/up ordinal parity: all compute threads stored h
   // ring entries: {queue position, then (before the unit's last stage lands)
   // the epilogue constants: global scale bits x2, any token prescaled}
-  int4* uent = reinterpret_cast<int4*>(uempty + kDecUnitRing);
+  int4* uent = reinterpret_cast<int4*>(hpub + 2);
   int4* udesc = uent + kDecUnitRing;   // [kDecUnitRing] the unit's descriptor, read once by the producer
-  int* abort_flag = reinterpret_cast<int*>(udesc + kDecUnitRing);
+  int* hcount = reinterpret_cast<int*>(udesc + kDecUnitRing);   // [2] warps that finished their h rows
+  int* abort_flag = hcount + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kDecStages; ++i) { mbar_init(&full[i], 2); mbar_init(&empty[i], 16); }
-    for (int i = 0; i < kDecUnitRing; ++i) { mbar_init(&ufull[i], 1); mbar_init(&uempty[i], 17); }
+    for (int i = 0; i < kDecUnitRing; ++i) { mbar_init(&ufull[i], 1); mbar_init(&uempty[i], 18); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&hpub[i], 512); hcount[i] = 0; }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -378,12 +385,18 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
     if (lane == 0) {
       uint32_t si = 0;
       bool ok = true;
+      // The next unit is taken from the queue (and its descriptor fetched)
+      // while the current one's stages are issued, so that the global
+      // round trips do not open a gap in the weight stream; it is handed to
+      // the consumers only once the ring has room for it.
+      int next_q = atomicAdd(p.queue, 1);
+      int4 next_raw = next_q < ntot ? unit_desc(p, next_q, n1) : make_int4(0, 0, 0, 0);
       for (int j = 0; ok; ++j) {
-        const int us = j % kDecUnitRing;   // take a unit only once there is room to hold it
+        const int us = j % kDecUnitRing;
         if (!(ok = ab.wait(&uempty[us], ((j / kDecUnitRing) & 1) ^ 1, kTagUnit, j, -3))) break;
-        int q = atomicAdd(p.queue, 1);
-        if (q >= ntot) q = -1;
-        const int4 raw = q >= 0 ? unit_desc(p, q, n1) : make_int4(0, 0, 0, 0);
+        const int q = next_q < ntot ? next_q : -1;
+        const int4 raw = next_raw;
+        if (q >= 0) next_q = atomicAdd(p.queue, 1);   // used after this unit's stages are issued
         udesc[us] = raw;
         uent[us].x = q;
         mbar_arrive(&ufull[us]);
@@ -409,6 +422,7 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
           tma_load_3d(st + kDecCodes, s0, &full[s], ws * 16, y0, slot);
           tma_load_3d(st + kDecCodes + 128 * 16, s1, &full[s], ws * 16, y1, slot);
         }
+        next_raw = next_q < ntot ? unit_desc(p, next_q, n1) : make_int4(0, 0, 0, 0);
       }
       dec_drain(full, si);
     }
@@ -441,9 +455,39 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
       }
       dec_drain(full, si);
     }
+  } else if (warp == 18) {
+    // --------------------------------------------------- publisher ---
+    // For each gate/up unit: once all compute threads stored their h rows,
+    // add the number of warps that finished to the token tile's count with
+    // one release (down units' token loaders acquire it).  The ring slot is
+    // released only after publishing, which bounds how far the compute
+    // warps run ahead of this warp.
+    if (lane == 0) {
+      int ngu = 0;
+      for (int j = 0;; ++j) {
+        const int us = j % kDecUnitRing;
+        if (!ab.wait(&ufull[us], (j / kDecUnitRing) & 1, kTagUnit, j, -4)) break;
+        const int q = uent[us].x;
+        if (q < 0) { mbar_arrive(&uempty[us]); break; }
+        const DecUnit d = decode_unit(p, q, n1, udesc[us]);
+        if (d.gemm == 0) {
+          const int hb = ngu & 1;
+          if (!ab.wait(&hpub[hb], (ngu >> 1) & 1, kTagUnit, ngu, q)) break;
+          const int cnt = hcount[hb];
+          hcount[hb] = 0;
+          if (cnt) {
+            fence_proxy_async_global();
+            red_release_gpu_add(p.tile_done + d.tile, cnt);
+          }
+          ++ngu;
+        }
+        mbar_arrive(&uempty[us]);
+      }
+    }
   } else {
     // --------------------------------------------------- compute ---
     uint32_t si = 0;
+    int ngu = 0;
     for (int j = 0;; ++j) {
       const int us = j % kDecUnitRing;
       if (!__all_sync(0xFFFFFFFFu, ab.wait(&ufull[us], (j / kDecUnitRing) & 1, kTagUnit, j, -2))) break;
@@ -454,8 +498,10 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
         break;
       }
       const DecUnit d = decode_unit(p, q, n1, udesc[us]);
-      const bool ok = d.nr > 8 ? dec_unit<2>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], si, q, warp, lane)
-                               : dec_unit<1>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], si, q, warp, lane);
+      const int gu = d.gemm == 0 ? ngu++ : -1;
+      const bool ok =
+          d.nr > 8 ? dec_unit<2>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], hpub, hcount, gu, si, q, warp, lane)
+                   : dec_unit<1>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], hpub, hcount, gu, si, q, warp, lane);
       if (!ok) break;
     }
   }
