@@ -286,12 +286,12 @@ FT_API int ft_slot_inject_copy_failures(ft_slot_mgr* mgr, int count);
 enum {
   FT_KERNEL_ROUTE = 0,
   FT_KERNEL_PERMUTE = 1,
-  FT_KERNEL_SCHEDULE = 2,
+  FT_KERNEL_SCHEDULE = 2,     /* (work lists; now built inside the FT_KERNEL_PREP launch) */
   FT_KERNEL_GEMM_GATE_UP = 3, /* grouped gate/up GEMM + SwiGLU */
   FT_KERNEL_GEMM_DOWN = 4,    /* grouped down GEMM */
   FT_KERNEL_COMBINE = 5,
   FT_KERNEL_PACK = 6,
-  FT_KERNEL_PREP = 7,         /* activations to f16 (inside ft_moe_ffn_nvfp4) */
+  FT_KERNEL_PREP = 7,         /* work lists + activations to f16 (inside ft_moe_ffn_nvfp4) */
   FT_KERNEL_FFN_DECODE = 8,   /* decode variant: gate/up + SwiGLU + down in one launch */
   FT_KERNEL_KINDS = 9,
 };

@@ -11,7 +11,7 @@
 // straight into warp-level MMA fragments (mma.sync m16n8k16, f16 x f16 ->
 // fp32): 256 weights per instruction, and the tensor cores do the FMAs.
 //
-// Work units (built on the device by ffn_schedule_kernel), in one queue:
+// Work units (built on the device by ffn_prep_kernel), in one queue:
 //   gate/up unit: 128 features (their 128 gate rows and 128 up rows) of one
 //                 expert x one group of <= 16 token rows x a K range;
 //   down unit:    256 rows of the down matrix x the same token group x a K range.
@@ -71,7 +71,7 @@ constexpr int kTagDep = 9;
 
 struct DecodeParams {
   FfnParams g[2];      // [0] gate/up + SwiGLU (h out), [1] down (out_perm out)
-  int* queue;          // next queue position to take (zeroed by ffn_schedule_kernel)
+  int* queue;          // next queue position to take (zeroed by ffn_prep_kernel)
   int* tile_done;      // per token tile: gate/up epilogue warps (16 per m-tile) that published h
   int mt1;             // gate/up m-tiles (128 features) per token tile
   int mt2;             // down m-tiles (256 rows) per token tile
@@ -191,7 +191,6 @@ __device__ __forceinline__ void dec_stage(const uint8_t* st, int r_lo, int r_hi,
 // streams in, and handed over through the unit ring.
 struct DecConsts {
   float g0, g1;        // global scales: gate and up (gate/up unit) or down twice
-  int any_scaled;      // gate/up: some token row was prescaled to fit f16
 };
 
 __device__ __forceinline__ DecConsts dec_consts(const DecodeParams& p, const DecUnit& d) {
@@ -200,7 +199,6 @@ __device__ __forceinline__ DecConsts dec_consts(const DecodeParams& p, const Dec
   DecConsts c;
   c.g0 = __ldg(reinterpret_cast<const float*>(sbase + G.global_off[0]));
   c.g1 = __ldg(reinterpret_cast<const float*>(sbase + G.global_off[1]));
-  c.any_scaled = d.gemm == 0 ? *G.any_scaled : 0;
   return c;
 }
 
@@ -210,7 +208,7 @@ __device__ __forceinline__ DecConsts dec_consts(const DecodeParams& p, const Dec
 // outputs.
 template <int NT>
 __device__ __forceinline__ bool dec_epilogue(const DecodeParams& p, const DecUnit& d, const DecConsts& c, int w,
-                                             int lane, float (&acc)[NT][4]) {
+                                             int lane, float (&acc)[NT][4], const float (&ts)[NT][2]) {
   const FfnParams& G = p.g[d.gemm];
   const int g = lane >> 2, t = lane & 3;
   if (G.splits > 1) {
@@ -244,8 +242,8 @@ __device__ __forceinline__ bool dec_epilogue(const DecodeParams& p, const DecUni
       for (int e = 0; e < 2; ++e) {
         const int r = 8 * n + 2 * t + e;
         if (r < d.nr && f < G.M) {
-          const float ts = c.any_scaled ? __ldg(G.tokscale + __ldg(G.perm_src + d.rb + r) / G.k_top) : 1.0f;
-          store_out<2>(G.out, size_t(d.rb + r) * G.M + f, silu_mul(c.g0 * ts * acc[n][e], c.g1 * ts * acc[n][2 + e]));
+          store_out<2>(G.out, size_t(d.rb + r) * G.M + f,
+                       silu_mul(c.g0 * ts[n][e] * acc[n][e], c.g1 * ts[n][e] * acc[n][2 + e]));
         }
       }
   } else {
@@ -279,6 +277,15 @@ __device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem,
                          int gu, uint32_t& si, int q, int w, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int r_lo = dec_row_lo(d.gemm, w, g), r_hi = dec_row_hi(d.gemm, w, g);
+  // gate/up: the factors undoing the token rows' prescale, loaded now, used in the epilogue
+  float ts[NT][2];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = 8 * n + 2 * t + e;
+      ts[n][e] = d.gemm == 0 && r < d.nr ? __ldg(p.g[0].rowscale + d.rb + r) : 1.0f;
+    }
   float acc[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n)
@@ -295,11 +302,11 @@ __device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem,
   DecConsts c;   // written by the weight producer before the last stage (acquired above)
   {
     const int4 ce = *unit_ent;
-    c.g0 = __int_as_float(ce.y); c.g1 = __int_as_float(ce.z); c.any_scaled = ce.w;
+    c.g0 = __int_as_float(ce.y); c.g1 = __int_as_float(ce.z);
   }
   __syncwarp();
   if (lane == 0) mbar_arrive(unit_free);   // the queue may hand this CTA its next-but-one unit
-  const bool fin = dec_epilogue<NT>(p, d, c, w, lane, acc);
+  const bool fin = dec_epilogue<NT>(p, d, c, w, lane, acc, ts);
   if (d.gemm == 0) {   // gate/up: hand the h rows to the publisher
     __syncwarp();
     if (fin && lane == 0) atomicAdd(&hcount[gu & 1], 1);
@@ -356,7 +363,7 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
   uint64_t* uempty = ufull + kDecUnitRing;
   uint64_t* hpub = uempty + kDecUnitRing;   // [2] by gate/up ordinal parity: all compute threads stored h
   // ring entries: {queue position, then (before the unit's last stage lands)
-  // the epilogue constants: global scale bits x2, any token prescaled}
+  // the epilogue constants: global scale bits x2}
   int4* uent = reinterpret_cast<int4*>(hpub + 2);
   int4* udesc = uent + kDecUnitRing;   // [kDecUnitRing] the unit's descriptor, read once by the producer
   int* hcount = reinterpret_cast<int*>(udesc + kDecUnitRing);   // [2] warps that finished their h rows
@@ -414,7 +421,7 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
           const int s = si % kDecStages;
           if (!(ok = ab.wait(&empty[s], ((si / kDecStages) & 1) ^ 1, kTagWEmpty, si, q))) break;
           if (ws == d.ws1 - 1)   // published by this stage's arrival (release) to the compute warps
-            uent[us] = make_int4(q, __float_as_int(c.g0), __float_as_int(c.g1), c.any_scaled);
+            uent[us] = make_int4(q, __float_as_int(c.g0), __float_as_int(c.g1), 0);
           mbar_arrive_expect_tx(&full[s], kDecWStageBytes);
           uint8_t* st = smem + s * kDecStageBytes;
           tma_load_3d(st, c0, &full[s], ws * 128, y0, slot);

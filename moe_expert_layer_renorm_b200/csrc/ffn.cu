@@ -43,8 +43,7 @@ constexpr int kMatStageBytes = kCodesBytes + kScaleBytes;   // 18 KB, multiple o
 constexpr int kThreads = 512;
 
 struct FfnParams {
-  const float* tokscale;      // GEMM1: per-token factor undoing the f16 prescale of x
-  const int* any_scaled;      // GEMM1: nonzero when some token was prescaled
+  const float* rowscale;      // GEMM1: per permuted row, the factor undoing the f16 prescale of x; GEMM2: null
   const int32_t* perm_src;    // GEMM1: row -> pair (token = pair / k_top); GEMM2: null (row -> row)
   int k_top;
   int K;                      // reduction length
@@ -175,11 +174,10 @@ __device__ __forceinline__ void store_out(void* out, size_t idx, float v) {
   }
 }
 
-// Factor undoing the power-of-two prescale of token row `row` of a group
-// (GEMM1 only; 1 when no token needed a prescale).
+// Factor undoing the power-of-two prescale of permuted row `row` (GEMM1; 1
+// for GEMM2, whose input h carries no prescale).
 __device__ __forceinline__ float token_factor(const FfnParams& p, int row) {
-  if (p.perm_src == nullptr || *p.any_scaled == 0) return 1.0f;
-  return __ldg(p.tokscale + __ldg(p.perm_src + row) / p.k_top);
+  return p.rowscale != nullptr ? __ldg(p.rowscale + row) : 1.0f;
 }
 
 template <int NMAT, int BN, int WS, int BS, int AS, int DB>
@@ -398,7 +396,6 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
       float gsc[NMAT];
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) gsc[m] = __ldg(reinterpret_cast<const float*>(sbase + p.global_off[m]));
-      const int any_scaled = NMAT == 2 && p.perm_src != nullptr ? *p.any_scaled : 0;
       if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&d_full[ds], (di / DB) & 1, kTagDFull, di, u)))) break;
       tc_fence_after();
       const int n_eff = (nr + 15) & ~15;
@@ -407,6 +404,9 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
         uint32_t v[NMAT][16];
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) tmem_ld_32x32b_x16(tmem + lane_base + (ds * NMAT + m) * BN + n0, v[m]);
+        float ts[16];   // the 16 token rows' prescale factors, loaded while tensor memory is read
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ts[i] = NMAT == 2 && !split && n0 + i < nr ? token_factor(p, rb + n0 + i) : 1.0f;
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -419,8 +419,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
           } else if (feat < p.M) {
             float r;
             if (NMAT == 2) {
-              const float ts = any_scaled ? token_factor(p, rb + n) : 1.0f;
-              r = silu_mul(gsc[0] * ts * __uint_as_float(v[0][i]), gsc[NMAT - 1] * ts * __uint_as_float(v[NMAT - 1][i]));
+              r = silu_mul(gsc[0] * ts[i] * __uint_as_float(v[0][i]), gsc[NMAT - 1] * ts[i] * __uint_as_float(v[NMAT - 1][i]));
             } else {
               r = gsc[0] * __uint_as_float(v[0][i]);
             }
@@ -454,7 +453,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
             if (feat < p.M) {
               float r;
               if (NMAT == 2) {
-                const float ts = any_scaled ? token_factor(p, rb + n) : 1.0f;
+                const float ts = token_factor(p, rb + n);
                 r = silu_mul(gsc[0] * ts * acc[0], gsc[NMAT - 1] * ts * acc[NMAT - 1]);
               } else {
                 r = gsc[0] * acc[0];
@@ -478,24 +477,123 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
 
 // ------------------------------------------------------------ x to f16 ---
 
+// ------------------------------------------------------ prep kernel ---
+//
+// One launch, two independent jobs that both need only the permutation:
+//   blocks [0, nsched)   the two work lists and the counter resets
+//   blocks [nsched, ..)  the f16 activations in permuted row order
+struct PrepParams {
+  // work lists
+  const int32_t* offsets;
+  const int32_t* slot_table;
+  int E, num_slots, nsched;
+  int bn1, mt1, s1, bn2, mt2, s2;
+  int4* units1;
+  int4* units2;
+  int* counts;                 // [0] units of GEMM1, [1] of GEMM2, [3] decode unit queue
+  int* counters1;
+  int ncnt1;
+  int* counters2;
+  int ncnt2;
+  int* tile_done;
+  int ndone;
+  // activations
+  const uint4* x;
+  const int32_t* perm_src;
+  int P, k_top, H;
+  uint4* x_perm;
+  float* rowscale;
+};
+
+__device__ int block_exclusive_scan(int v, int* smem_warp_sums);
+
+// Work lists.  Unit u = ((tile * m_tiles) + m_tile) * splits + split, tiles
+// numbered in expert order, so the splits of one output tile are
+// consecutive.  Every schedule block derives the experts' first tiles (each
+// thread 4 experts, E <= 1024) and writes a strided share of the units, each
+// unit's expert found by binary search over the first tiles.
+__device__ void prep_schedule(const PrepParams& p, int b) {
+  __shared__ int warp_sums[32];
+  __shared__ int start1[kMaxExperts + 1], start2[kMaxExperts + 1];
+  __shared__ int s_rb[kMaxExperts], s_n[kMaxExperts], s_slot[kMaxExperts];
+  const int E = p.E;
+  int c1[4], c2[4], sum1 = 0, sum2 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 4 * threadIdx.x + i;
+    int n = 0, rb = 0, slot = 0;
+    if (e < E) {
+      rb = p.offsets[e];
+      n = p.offsets[e + 1] - rb;
+      if (n > 0) {
+        slot = p.slot_table[e];
+        if (slot < 0) { if (b == 0) set_device_status(FT_DEV_NOT_RESIDENT); n = 0; }
+        else if (slot >= p.num_slots) { if (b == 0) set_device_status(FT_DEV_BAD_INDEX); n = 0; }
+      }
+      s_rb[e] = rb;
+      s_n[e] = n;
+      s_slot[e] = slot;
+    }
+    c1[i] = (n + p.bn1 - 1) / p.bn1;
+    c2[i] = (n + p.bn2 - 1) / p.bn2;
+    sum1 += c1[i];
+    sum2 += c2[i];
+  }
+  int ex1 = block_exclusive_scan(sum1, warp_sums);
+  int ex2 = block_exclusive_scan(sum2, warp_sums);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 4 * threadIdx.x + i;
+    if (e < E) { start1[e] = ex1; start2[e] = ex2; }
+    ex1 += c1[i];
+    ex2 += c2[i];
+  }
+  if (threadIdx.x == blockDim.x - 1) { start1[E] = ex1; start2[E] = ex2; }   // the totals
+  __syncthreads();
+  const int stride = blockDim.x * p.nsched, first = threadIdx.x + blockDim.x * b;
+  auto fill = [&](const int* start, int bn, int mt, int sp, int4* units) {
+    const int total = start[E] * mt * sp;
+    for (int u = first; u < total; u += stride) {
+      const int tile = u / (mt * sp), rem = u - tile * (mt * sp);
+      int lo = 0, hi = E;                 // last expert whose first tile is <= tile
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (start[mid] <= tile) lo = mid; else hi = mid;
+      }
+      const int t = tile - start[lo];
+      units[u] = make_int4(lo | (s_slot[lo] << 10), rem / sp, s_rb[lo] + t * bn,
+                           min(bn, s_n[lo] - t * bn) | ((rem % sp) << 16));
+    }
+    return total;
+  };
+  const int total1 = fill(start1, p.bn1, p.mt1, p.s1, p.units1);
+  const int total2 = fill(start2, p.bn2, p.mt2, p.s2, p.units2);
+  if (b == 0 && threadIdx.x == 0) {
+    p.counts[0] = total1;
+    p.counts[1] = total2;
+    p.counts[2] = 0;
+    p.counts[3] = 0;   // decode unit queue
+  }
+  for (int i = first; i < p.ncnt1; i += stride) p.counters1[i] = 0;
+  for (int i = first; i < p.ncnt2; i += stride) p.counters2[i] = 0;
+  for (int i = first; i < p.ndone; i += stride) p.tile_done[i] = 0;
+}
+
 // One warp per permuted row r (token t = perm_src[r] / k): writes
-// x_perm[r] = f16(x[t] * 2^-s_t) and tokscale[t] = 2^s_t, with s_t >= 0 the
+// x_perm[r] = f16(x[t] * 2^-s_t) and rowscale[r] = 2^s_t, with s_t >= 0 the
 // smallest shift that brings max|x[t]| below 2^15.  The f16 conversion is
 // then exact for every element of the row within a factor 2^32 of the row's
 // largest magnitude (bf16 has 8 significant bits, f16 subnormals reach
 // 2^-24); smaller elements round with an absolute error below 2^-41 max|x[t]|.
 // Rows in permuted order make each expert group's tokens one contiguous
 // block, so the GEMM loads them as plain tiles.
-__global__ void __launch_bounds__(256) prep_x_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_src,
-                                                     int P, int k_top, int H, uint4* __restrict__ x_perm,
-                                                     float* __restrict__ tokscale, int* __restrict__ any_scaled) {
-  pdl_enter();
+__device__ void prep_rows(const PrepParams& p, int b) {
   const int lane = threadIdx.x & 31;
-  const int r = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  if (r >= P) return;
-  const int t = __ldg(perm_src + r) / k_top;
-  const int nv = H / 8;
-  const uint4* row = x + size_t(t) * nv;
+  const int r = b * (blockDim.x / 32) + threadIdx.x / 32;
+  if (r >= p.P) return;
+  const int t = __ldg(p.perm_src + r) / p.k_top;
+  const int nv = p.H / 8;
+  const uint4* row = p.x + size_t(t) * nv;
   float m = 0.0f;
   for (int c = lane; c < nv; c += 32) {
     const uint4 v = __ldg(row + c);
@@ -515,11 +613,8 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const uint4* __restrict__ x
     set_device_status(FT_DEV_F16_RANGE);         // inf or nan input
   }
   const float f = ldexpf(1.0f, -shift);
-  if (lane == 0) {
-    tokscale[t] = ldexpf(1.0f, shift);           // every row of token t writes the same value
-    if (shift) atomicOr(any_scaled, 1);
-  }
-  uint4* out = x_perm + size_t(r) * nv;
+  if (lane == 0) p.rowscale[r] = ldexpf(1.0f, shift);
+  uint4* out = p.x_perm + size_t(r) * nv;
   for (int c = lane; c < nv; c += 32) {
     const uint4 v = __ldg(row + c);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -533,69 +628,10 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const uint4* __restrict__ x
   }
 }
 
-// ----------------------------------------------------------- schedule ---
-
-__device__ int block_exclusive_scan(int v, int* smem_warp_sums);
-
-// Builds both GEMMs' work lists from the expert offsets (one CTA; E <= 1024).
-// Unit u = ((tile * m_tiles) + m_tile) * splits + split, tiles numbered in
-// expert order, so the splits of one output tile are consecutive.
-__global__ void __launch_bounds__(1024) ffn_schedule_kernel(
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ slot_table, int E, int num_slots,
-    int bn1, int mt1, int s1, int bn2, int mt2, int s2, int4* __restrict__ units1, int4* __restrict__ units2,
-    int* __restrict__ counts, int* __restrict__ counters1, int ncnt1, int* __restrict__ counters2, int ncnt2,
-    int* __restrict__ tile_done, int ndone) {
+__global__ void __launch_bounds__(256) ffn_prep_kernel(const PrepParams p) {
   pdl_enter();
-  __shared__ int warp_sums[32];
-  __shared__ int start1[kMaxExperts + 1], start2[kMaxExperts + 1];   // first tile of each expert
-  __shared__ int s_rb[kMaxExperts], s_n[kMaxExperts], s_slot[kMaxExperts];
-  const int e = threadIdx.x;
-  int n = 0, rb = 0, slot = 0;
-  if (e < E) {
-    rb = offsets[e];
-    n = offsets[e + 1] - rb;
-    if (n > 0) {
-      slot = slot_table[e];
-      if (slot < 0) { set_device_status(FT_DEV_NOT_RESIDENT); n = 0; }
-      else if (slot >= num_slots) { set_device_status(FT_DEV_BAD_INDEX); n = 0; }
-    }
-    s_rb[e] = rb;
-    s_n[e] = n;
-    s_slot[e] = slot;
-  }
-  const int t1 = (n + bn1 - 1) / bn1, t2 = (n + bn2 - 1) / bn2;
-  const int ex1 = block_exclusive_scan(t1, warp_sums);
-  const int ex2 = block_exclusive_scan(t2, warp_sums);
-  if (e < E) { start1[e] = ex1; start2[e] = ex2; }
-  if (e == E - 1) { start1[E] = ex1 + t1; start2[E] = ex2 + t2; }
-  __syncthreads();
-  // every thread writes units of every expert: u -> (tile, m-tile, split),
-  // the tile's expert by binary search over the experts' first tiles
-  auto fill = [&](const int* start, int bn, int mt, int sp, int4* units) {
-    const int total = start[E] * mt * sp;
-    for (int u = threadIdx.x; u < total; u += blockDim.x) {
-      const int tile = u / (mt * sp), rem = u - tile * (mt * sp);
-      int lo = 0, hi = E;                 // last expert whose first tile is <= tile
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (start[mid] <= tile) lo = mid; else hi = mid;
-      }
-      const int t = tile - start[lo];
-      units[u] = make_int4(lo | (s_slot[lo] << 10), rem / sp, s_rb[lo] + t * bn,
-                           min(bn, s_n[lo] - t * bn) | ((rem % sp) << 16));
-    }
-    return total;
-  };
-  const int total1 = fill(start1, bn1, mt1, s1, units1);
-  const int total2 = fill(start2, bn2, mt2, s2, units2);
-  if (threadIdx.x == 0) {
-    counts[0] = total1;
-    counts[1] = total2;
-  }
-  if (threadIdx.x == 0) { counts[2] = 0; counts[3] = 0; }   // any token prescaled; unit queue
-  for (int i = threadIdx.x; i < ncnt1; i += blockDim.x) counters1[i] = 0;
-  for (int i = threadIdx.x; i < ncnt2; i += blockDim.x) counters2[i] = 0;
-  for (int i = threadIdx.x; i < ndone; i += blockDim.x) tile_done[i] = 0;
+  if (int(blockIdx.x) < p.nsched) prep_schedule(p, blockIdx.x);
+  else prep_rows(p, blockIdx.x - p.nsched);
 }
 
 }  // namespace ftmoe

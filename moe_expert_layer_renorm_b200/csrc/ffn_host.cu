@@ -17,7 +17,7 @@ struct FfnPlan {
   int mt1, mt2, nkw1, nkw2, nkc1, nkc2;
   long long max_tiles1, max_tiles2;
   // workspace layout (byte offsets)
-  size_t off_h, off_x16, off_tokscale, off_units1, off_units2, off_counts, off_cnt1, off_cnt2, off_done, off_part1,
+  size_t off_h, off_x16, off_rowscale, off_units1, off_units2, off_counts, off_cnt1, off_cnt2, off_done, off_part1,
       off_part2, total;
   long long max_units1, max_units2;
   int cnt_per;
@@ -108,7 +108,7 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   size_t o = 0;
   pl.off_h = o;       o = align256(o + size_t(P) * I * 2);
   pl.off_x16 = o;     o = align256(o + size_t(P) * H * 2);   // f16 activations, permuted rows
-  pl.off_tokscale = o; o = align256(o + size_t(T) * 4);
+  pl.off_rowscale = o; o = align256(o + size_t(P) * 4);
   pl.off_units1 = o;  o = align256(o + size_t(pl.max_units1) * 16);
   pl.off_units2 = o;  o = align256(o + size_t(pl.max_units2) * 16);
   pl.off_counts = o;  o = align256(o + 16);   // [0] units of GEMM1, [1] of GEMM2, [2] any token prescaled, [3] queue
@@ -223,20 +223,35 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   int* cnt2 = reinterpret_cast<int*>(w + pl.off_cnt2);
   __half* h = reinterpret_cast<__half*>(w + pl.off_h);
   __half* x16 = reinterpret_cast<__half*>(w + pl.off_x16);
-  float* tokscale = reinterpret_cast<float*>(w + pl.off_tokscale);
+  float* rowscale = reinterpret_cast<float*>(w + pl.off_rowscale);
   cudaError_t err;
   {
-    ProfileScope prof(FT_KERNEL_SCHEDULE, s);
-    err = launch_pdl(ffn_schedule_kernel, dim3(1), dim3(1024), 0, s, offsets, slot_table, E, L.num_slots, pl.g1.bn,
-                     pl.mt1, pl.g1.splits, pl.g2.bn, pl.mt2, pl.g2.splits, units1, units2, counts, cnt1,
-                     int(pl.max_tiles1 * pl.mt1 * pl.cnt_per), cnt2, int(pl.max_tiles2 * pl.mt2 * pl.cnt_per),
-                     reinterpret_cast<int*>(w + pl.off_done), pl.decode ? int(pl.max_tiles1) : 0);
-  }
-  if (err != cudaSuccess) return err;
-  {
+    PrepParams pp{};
+    pp.offsets = offsets;
+    pp.slot_table = slot_table;
+    pp.E = E;
+    pp.num_slots = L.num_slots;
+    pp.nsched = int(std::min<long long>(32, std::max<long long>(1, (pl.max_units1 + pl.max_units2) / 4096)));
+    pp.bn1 = pl.g1.bn; pp.mt1 = pl.mt1; pp.s1 = pl.g1.splits;
+    pp.bn2 = pl.g2.bn; pp.mt2 = pl.mt2; pp.s2 = pl.g2.splits;
+    pp.units1 = units1;
+    pp.units2 = units2;
+    pp.counts = counts;
+    pp.counters1 = cnt1;
+    pp.ncnt1 = int(pl.max_tiles1 * pl.mt1 * pl.cnt_per);
+    pp.counters2 = cnt2;
+    pp.ncnt2 = int(pl.max_tiles2 * pl.mt2 * pl.cnt_per);
+    pp.tile_done = reinterpret_cast<int*>(w + pl.off_done);
+    pp.ndone = pl.decode ? int(pl.max_tiles1) : 0;
+    pp.x = static_cast<const uint4*>(x);
+    pp.perm_src = perm_src;
+    pp.P = T * k;
+    pp.k_top = k;
+    pp.H = H;
+    pp.x_perm = reinterpret_cast<uint4*>(x16);
+    pp.rowscale = rowscale;
     ProfileScope prof(FT_KERNEL_PREP, s);
-    err = launch_pdl(prep_x_kernel, dim3((T * k + 7) / 8), dim3(256), 0, s, static_cast<const uint4*>(x), perm_src,
-                     T * k, k, H, reinterpret_cast<uint4*>(x16), tokscale, counts + 2);
+    err = launch_pdl(ffn_prep_kernel, dim3(pp.nsched + (T * k + 7) / 8), dim3(256), 0, s, pp);
   }
   if (err != cudaSuccess) return err;
 
@@ -247,8 +262,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
     return cudaErrorInvalidValue;
   }
   FfnParams p1{};
-  p1.tokscale = tokscale;
-  p1.any_scaled = counts + 2;
+  p1.rowscale = rowscale;
   p1.perm_src = perm_src;
   p1.k_top = k;
   p1.K = H;
@@ -271,6 +285,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
 
   FfnParams p2 = p1;
   p2.perm_src = nullptr;
+  p2.rowscale = nullptr;
   p2.K = I;
   p2.M = H;
   p2.nkw = pl.nkw2;
