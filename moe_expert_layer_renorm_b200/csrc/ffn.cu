@@ -285,17 +285,19 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
           if (!(ok = ab.wait(&a_full[as], (q / AS) & 1, kTagAFull, q, u))) break;
           if (!(ok = ab.wait(&b_full[bs], (q / BS) & 1, kTagBFull, q, u))) break;
           tc_fence_after();
-          const uint32_t b_addr = smem_u32(b_smem + bs * Cfg::kBStageBytes);
+          // every operand address first, then the MMAs back to back: the
+          // issuing thread's own instructions between MMAs cost tensor time
+          const uint64_t bd = make_sdesc_sw128(smem_u32(b_smem + bs * Cfg::kBStageBytes));
+          const uint32_t d0 = tmem + ds * NMAT * BN;
+          const uint32_t a0 = tmem + Cfg::kDCols + as * NMAT * 32;
+          const uint32_t acc0 = c > kc0 ? 1u : 0u;
 #pragma unroll
-          for (int j = 0; j < kKC / 16; ++j) {
-            const uint64_t bdesc = make_sdesc_sw128(b_addr + 32 * j);
+          for (int m = 0; m < NMAT; ++m) mma_ts_f16(d0 + m * BN, a0 + m * 32, bd, idesc, acc0);
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-              const uint32_t d_addr = tmem + (ds * NMAT + m) * BN;
-              const uint32_t a_addr = tmem + Cfg::kDCols + (as * NMAT + m) * 32 + 8 * j;
-              mma_ts_f16(d_addr, a_addr, bdesc, idesc, (c > kc0 || j > 0) ? 1u : 0u);
-            }
-          }
+          for (int j = 1; j < kKC / 16; ++j)
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)   // K slice j: +32 bytes of B (+2 in the descriptor's address field)
+              mma_ts_f16_acc(d0 + m * BN, a0 + m * 32 + 8 * j, bd + uint64_t(2 * j), idesc);
           issued = true;
           mma_commit(&a_empty[as]);
           mma_commit(&b_empty[bs]);

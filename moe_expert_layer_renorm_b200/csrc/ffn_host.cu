@@ -43,6 +43,12 @@ static int choose_splits(double units_est, int nkw, int num_sms, double split_co
   return best;
 }
 
+// Prefill tile shapes <token rows (MMA N), weight stages, token stages, A
+// stages, accumulator buffers> of the two tcgen05 GEMMs.  Tensor memory
+// holds DB * NMAT * BN accumulator columns plus AS * NMAT * 32 for A.
+constexpr int kPreBN1 = 128, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 4, kPreDB1 = 1;
+constexpr int kPreBN2 = 128, kPreWS2 = 3, kPreBS2 = 6, kPreAS2 = 4, kPreDB2 = 2;
+
 // Decode split-K: the smallest divisor of the K-stage count that gives every
 // SM a unit (a dynamic queue balances the rest, so waves do not matter).
 static int decode_splits(double units_est, int nkw, int num_sms, int* sps_out) {
@@ -79,8 +85,8 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
     pl.g1 = {kDecBN, 1, 0, 4, 0, 0, 0};
     pl.g2 = {kDecBN, 1, 0, 4, 0, 0, 0};
   } else {
-    pl.g1 = {128, 1, 0, 3, 4, 4, 1};
-    pl.g2 = {128, 1, 0, 3, 6, 4, 2};
+    pl.g1 = {kPreBN1, 1, 0, kPreWS1, kPreBS1, kPreAS1, kPreDB1};
+    pl.g2 = {kPreBN2, 1, 0, kPreWS2, kPreBS2, kPreAS2, kPreDB2};
   }
   const double tiles_per_expert1 = std::max(1.0, ceil(mean_rows / pl.g1.bn));
   const double tiles_per_expert2 = std::max(1.0, ceil(mean_rows / pl.g2.bn));
@@ -312,8 +318,9 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
     const int grid = int(std::min<long long>(num_sms, pl.max_units1 + pl.max_units2));
     err = launch_decode(dp, grid, tmc, tms, tm_x, tm_h, s);
   } else {
-    err = launch_gemm<2, 128, 3, 4, 4, 1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
-    if (err == cudaSuccess) err = launch_gemm<1, 128, 3, 6, 4, 2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
+    err = launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    if (err == cudaSuccess)
+      err = launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   }
   return err;
 }
