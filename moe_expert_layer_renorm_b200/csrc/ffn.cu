@@ -131,6 +131,10 @@ __device__ __forceinline__ void dequant_chunk(const uint4& c0, const uint4& c1, 
 // Barrier kinds, recorded with a wait timeout.
 enum : int { kTagWEmpty = 1, kTagWFull, kTagBEmpty, kTagBFull, kTagAEmpty, kTagAFull, kTagDEmpty, kTagDFull };
 
+// Named barrier (id 0 is __syncthreads) shared by the MMA warp and the
+// operand-waiter warp.
+constexpr int kBarHandoff = 1;
+
 struct Abort {
   volatile int* flag;
   __device__ bool wait(uint64_t* bar, uint32_t parity, int tag = 0, long long counter = 0,
@@ -203,6 +207,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
   uint64_t* drain_bar = d_empty + DB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* handoff = abort_flag + 1;   // [2]: waiter -> MMA warp, per chunk (by parity): 1 go, 0 stop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -269,24 +274,27 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer ---
-    if (lane == 0) {
-      uint32_t q = 0, di = 0;
-      bool ok = true, issued = false;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++di) {
-        int e, mt, rb, nr, ws0, ws1, kc0, kc1;
-        unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
-        const int ds = di % DB;
-        if (!(ok = ab.wait(&d_empty[ds], ((di / DB) & 1) ^ 1, kTagDEmpty, di, u))) break;
-        tc_fence_after();
-        const int n_eff = (nr + 15) & ~15;
-        const uint32_t idesc = make_idesc_f16(128, n_eff, /*f16 operands=*/true);
-        for (int c = kc0; c < kc1; ++c, ++q) {
-          const int as = q % AS, bs = q % BS;
-          if (!(ok = ab.wait(&a_full[as], (q / AS) & 1, kTagAFull, q, u))) break;
-          if (!(ok = ab.wait(&b_full[bs], (q / BS) & 1, kTagBFull, q, u))) break;
+    // Waits on no mbarrier inside the loop: an mbarrier wait (or a polled
+    // flag) in the issuing thread leaves the tensor pipe idle for a few
+    // hundred cycles even when the operands are already in place.  Warp 3
+    // does the waiting; the two warps meet at a named barrier once per chunk,
+    // with warp 3 one chunk ahead, and warp 3 leaves its verdict in
+    // handoff[q & 1] before it arrives.  Both warps run the same chunk
+    // sequence and leave at the same chunk, so every barrier phase completes.
+    uint32_t q = 0, di = 0;
+    bool ok = true, issued = false;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++di) {
+      int e, mt, rb, nr, ws0, ws1, kc0, kc1;
+      unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+      const int ds = di % DB;
+      const int n_eff = (nr + 15) & ~15;
+      const uint32_t idesc = make_idesc_f16(128, n_eff, /*f16 operands=*/true);
+      for (int c = kc0; c < kc1; ++c, ++q) {
+        named_bar_sync(kBarHandoff, 64);
+        if (!(ok = *reinterpret_cast<volatile int*>(handoff + (q & 1)) != 0)) break;
+        if (lane == 0) {
           tc_fence_after();
-          // every operand address first, then the MMAs back to back: the
-          // issuing thread's own instructions between MMAs cost tensor time
+          const int as = q % AS, bs = q % BS;
           const uint64_t bd = make_sdesc_sw128(smem_u32(b_smem + bs * Cfg::kBStageBytes));
           const uint32_t d0 = tmem + ds * NMAT * BN;
           const uint32_t a0 = tmem + Cfg::kDCols + as * NMAT * 32;
@@ -298,38 +306,39 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)   // K slice j: +32 bytes of B (+2 in the descriptor's address field)
               mma_ts_f16_acc(d0 + m * BN, a0 + m * 32 + 8 * j, bd + uint64_t(2 * j), idesc);
-          issued = true;
           mma_commit(&a_empty[as]);
           mma_commit(&b_empty[bs]);
         }
-        if (!ok) break;
-        mma_commit(&d_full[ds]);
+        issued = true;
+        __syncwarp();
       }
-      if (issued) {   // drain: every MMA this thread issued has completed
-        mma_commit(drain_bar);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
-      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(&d_full[ds]);
+      __syncwarp();
+    }
+    if (issued && lane == 0) {   // drain: every MMA this thread issued has completed
+      mma_commit(drain_bar);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
     }
   } else if (warp == 2) {
     // --------------------------------------------- B (token) producer ---
-    // Lane 0 issues one 16-row TMA tile per 16 rows for every 64-K chunk.
-    // Rows past the group end but below the MMA's N are other groups' rows
-    // (or zero fill past the last row): finite, and their results are never
-    // stored.
+    // Lane 0 issues one BN-row TMA box per 64-K chunk (one large box keeps
+    // the copy engine's per-box cost off the critical path; 16-row boxes
+    // were several times slower).  Rows past the group end are other
+    // groups' rows (or zero fill past the last row): finite, and their
+    // results are never stored.
     uint32_t q = 0;
     bool ok = true;
     if (lane == 0) {
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int e, mt, rb, nr, ws0, ws1, kc0, kc1;
         unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
-        const int n_eff = (nr + 15) & ~15;
         for (int c = kc0; c < kc1; ++c, ++q) {
           const int bs = q % BS;
           if (!(ok = ab.wait(&b_empty[bs], ((q / BS) & 1) ^ 1, kTagBEmpty, q, u))) break;
-          mbar_arrive_expect_tx(&b_full[bs], uint32_t(n_eff) * 128u);
-          uint8_t* dst = b_smem + bs * Cfg::kBStageBytes;
-          for (int n = 0; n < n_eff; n += 16) tma_load_2d(dst + n * 128, &tm_act, &b_full[bs], c * kKC, rb + n);
+          mbar_arrive_expect_tx(&b_full[bs], uint32_t(BN) * 128u);
+          tma_load_2d(b_smem + bs * Cfg::kBStageBytes, &tm_act, &b_full[bs], c * kKC, rb);
         }
       }
       for (uint32_t j = (q > BS ? q - BS : 0); j < q; ++j) {   // drain
@@ -338,8 +347,31 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
       }
     }
   } else if (warp == 3) {
-    // idle: keeps the dequantising warps at warp indices 4..11, so that warp % 4
-    // names the 32-lane quarter of tensor memory each of them may access
+    // ---------------------------------------------- operand waiter ---
+    // Lane 0 waits, in the MMA warp's order, for each unit's accumulator
+    // buffer to be drained and for each chunk's A (dequantised weights) and B
+    // (tokens) to be in place; the warp then meets the MMA warp at the named
+    // barrier.  Its place at warp index 3 also keeps the dequantising warps at
+    // 4..11, so that warp % 4 names the 32-lane quarter of tensor memory each
+    // of them may access.
+    uint32_t q = 0, di = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++di) {
+      int e, mt, rb, nr, ws0, ws1, kc0, kc1;
+      unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+      const int ds = di % DB;
+      for (int c = kc0; c < kc1; ++c, ++q) {
+        if (lane == 0) {
+          if (c == kc0) ok = ab.wait(&d_empty[ds], ((di / DB) & 1) ^ 1, kTagDEmpty, di, u);
+          ok = ok && ab.wait(&a_full[q % AS], (q / AS) & 1, kTagAFull, q, u);
+          ok = ok && ab.wait(&b_full[q % BS], (q / BS) & 1, kTagBFull, q, u);
+          *reinterpret_cast<volatile int*>(handoff + (q & 1)) = ok ? 1 : 0;
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        named_bar_sync(kBarHandoff, 64);
+        if (!ok) break;
+      }
+    }
   } else if (warp >= 4 && warp < 12) {
     // -------------------------------------------------- dequantise ---
     const int g = (warp - 4) >> 2;            // warpgroup: even / odd chunks
@@ -398,40 +430,68 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
       float gsc[NMAT];
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) gsc[m] = __ldg(reinterpret_cast<const float*>(sbase + p.global_off[m]));
+      const bool split = p.splits > 1;
+      // prescale factors of the unit's token rows, one coalesced load per 32
+      // rows issued before the accumulators are ready; lane j of group g holds
+      // row 32 g + j and the block loop broadcasts them with shuffles
+      constexpr int kGroups = (BN + 31) / 32;
+      float tsl[kGroups];
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g)
+        tsl[g] = NMAT == 2 && !split && g * 32 + lane < nr ? token_factor(p, rb + g * 32 + lane) : 1.0f;
       if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&d_full[ds], (di / DB) & 1, kTagDFull, di, u)))) break;
       tc_fence_after();
       const int n_eff = (nr + 15) & ~15;
-      const bool split = p.splits > 1;
-      for (int n0 = 0; n0 < n_eff; n0 += 16) {
-        uint32_t v[NMAT][16];
+      // 16-column blocks, the tensor-memory load of block b + 1 in flight while
+      // block b is computed; the accumulator buffer is handed back as soon as
+      // its last block has been loaded
+      uint32_t v[2][NMAT][16];
+      const uint32_t dcol = tmem + lane_base + ds * NMAT * BN;
+      if (n_eff > 0) {
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m) tmem_ld_32x32b_x16(tmem + lane_base + (ds * NMAT + m) * BN + n0, v[m]);
-        float ts[16];   // the 16 token rows' prescale factors, loaded while tensor memory is read
+        for (int m = 0; m < NMAT; ++m) tmem_ld_32x32b_x16(dcol + m * BN, v[0][m]);
+      }
+      bool released = false;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ts[i] = NMAT == 2 && !split && n0 + i < nr ? token_factor(p, rb + n0 + i) : 1.0f;
+      for (int bk = 0; bk < BN / 16; ++bk) {
+        const int n0 = bk * 16;
+        if (n0 >= n_eff) break;
         tmem_wait_ld();
+        if (n0 + 16 < n_eff) {
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) tmem_ld_32x32b_x16(dcol + m * BN + n0 + 16, v[(bk + 1) & 1][m]);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&d_empty[ds]);
+          released = true;
+        }
+        const uint32_t (&w)[NMAT][16] = v[bk & 1];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int n = n0 + i;
+          const float ts = __shfl_sync(0xFFFFFFFFu, tsl[bk >> 1], (bk & 1) * 16 + i);
           if (n >= nr) break;
           if (split) {
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
-              p.partials[(size_t(u) * NMAT + m) * 128 * BN + size_t(n) * 128 + row] = __uint_as_float(v[m][i]);
+              p.partials[(size_t(u) * NMAT + m) * 128 * BN + size_t(n) * 128 + row] = __uint_as_float(w[m][i]);
           } else if (feat < p.M) {
             float r;
             if (NMAT == 2) {
-              r = silu_mul(gsc[0] * ts[i] * __uint_as_float(v[0][i]), gsc[NMAT - 1] * ts[i] * __uint_as_float(v[NMAT - 1][i]));
+              r = silu_mul(gsc[0] * ts * __uint_as_float(w[0][i]), gsc[NMAT - 1] * ts * __uint_as_float(w[NMAT - 1][i]));
             } else {
-              r = gsc[0] * __uint_as_float(v[0][i]);
+              r = gsc[0] * __uint_as_float(w[0][i]);
             }
             store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&d_empty[ds]);
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_empty[ds]);
+      }
       if (split) {
         // this warp's 32 rows: the last of the `splits` warps to arrive sums
         // the partials in split order and writes the result

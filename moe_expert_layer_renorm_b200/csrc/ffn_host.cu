@@ -46,8 +46,8 @@ static int choose_splits(double units_est, int nkw, int num_sms, double split_co
 // Prefill tile shapes <token rows (MMA N), weight stages, token stages, A
 // stages, accumulator buffers> of the two tcgen05 GEMMs.  Tensor memory
 // holds DB * NMAT * BN accumulator columns plus AS * NMAT * 32 for A.
-constexpr int kPreBN1 = 128, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 4, kPreDB1 = 1;
-constexpr int kPreBN2 = 128, kPreWS2 = 3, kPreBS2 = 6, kPreAS2 = 4, kPreDB2 = 2;
+constexpr int kPreBN1 = 96, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 2, kPreDB1 = 2;
+constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 6, kPreAS2 = 4, kPreDB2 = 2;
 
 // Decode split-K: the smallest divisor of the K-stage count that gives every
 // SM a unit (a dynamic queue balances the rest, so waves do not matter).
@@ -171,8 +171,8 @@ static bool make_weight_maps(const uint8_t* pool, const ft_nvfp4_slot_layout& L,
 }
 
 // Activation rows (bf16 [rows, K]) as the MMA's B operand, 64-column (128-byte)
-// boxes with the 128-byte swizzle: one-row boxes for tile::gather4, or
-// 16-row boxes for contiguous rows.
+// boxes with the 128-byte swizzle: box_rows contiguous rows (the decode
+// kernel's token tile, or a prefill GEMM's whole BN-row token tile).
 static bool make_act_map(const void* base, int rows, int K, int box_rows, CUtensorMap* m) {  // f16 rows
   auto enc = tensor_map_encoder();
   if (!enc) return false;
@@ -262,8 +262,8 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   if (err != cudaSuccess) return err;
 
   CUtensorMap tm_x, tm_h;
-  const int act_box = pl.decode ? kDecBN : 16;
-  if (!make_act_map(x16, T * k, H, act_box, &tm_x) || !make_act_map(h, T * k, I, act_box, &tm_h)) {
+  if (!make_act_map(x16, T * k, H, pl.decode ? kDecBN : kPreBN1, &tm_x) ||
+      !make_act_map(h, T * k, I, pl.decode ? kDecBN : kPreBN2, &tm_h)) {
     *why = "cuTensorMapEncodeTiled failed for the activations";
     return cudaErrorInvalidValue;
   }
