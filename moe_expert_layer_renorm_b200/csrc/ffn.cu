@@ -35,8 +35,7 @@
 namespace ftmoe {
 
 constexpr int kKW = 256;            // K per weight stage (128 bytes of codes per row)
-constexpr int kKC = 64;             // K per chunk (one 128-byte swizzle atom of bf16)
-constexpr int kCPW = kKW / kKC;     // chunks per weight stage
+constexpr int kAtomK = 64;          // K of one 128-byte swizzle atom of f16 (one token-tile box)
 constexpr int kCodesBytes = 128 * 128;
 constexpr int kScaleBytes = 128 * 16;
 constexpr int kMatStageBytes = kCodesBytes + kScaleBytes;   // 18 KB, multiple of 1024
@@ -49,7 +48,7 @@ struct FfnParams {
   int K;                      // reduction length
   int M;                      // output features (rows of the weight matrices)
   int nkw;                    // ceil(K / kKW)
-  int nkc;                    // K / kKC
+  int nkc;                    // ceil(K / KC): chunks of the kernel's chunk size
   int splits;                 // split-K factor
   int stages_per_split;
   const int4* units;          // {expert | slot << 10, m_tile, row_begin, n_rows | split << 16}
@@ -63,15 +62,23 @@ struct FfnParams {
   int* counters;              // split-K arrival counters, 4 per (tile, m_tile): one per epilogue warp
 };
 
-template <int NMAT, int BN, int WS, int BS, int AS, int DB>
+// KC: K per chunk (64 or 128), the unit of one dequantised A slot, one
+// token stage and one operand hand-over to the MMA warp.  A chunk of 128
+// halves the per-chunk costs (barriers, hand-over, commits) per MMA.
+template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC>
 struct FfnCfg {
+  static constexpr int kAtoms = KC / kAtomK;                 // swizzle atoms (token boxes) per chunk
+  static constexpr int kCPW = kKW / KC;                      // chunks per weight stage
+  static constexpr int kACols = KC / 2;                      // tensor-memory columns of one matrix's A slot
   static constexpr int kWBytes = WS * NMAT * kMatStageBytes;
-  static constexpr int kBStageBytes = BN * 128;
+  static constexpr int kBAtomBytes = BN * 128;
+  static constexpr int kBStageBytes = kAtoms * kBAtomBytes;
   static constexpr int kBBytes = BS * kBStageBytes;
   static constexpr int kNumBars = 2 * WS + 2 * BS + 2 * AS + 2 * DB + 1;
   static constexpr int kSmemBytes = 1024 /*align slack*/ + kWBytes + kBBytes + BN * 4 + kNumBars * 8 + 64;
   static constexpr int kDCols = DB * NMAT * BN;
-  static constexpr int kTmemCols = kDCols + AS * NMAT * 32;
+  static constexpr int kTmemCols = kDCols + AS * NMAT * kACols;
+  static_assert(KC == 64 || KC == 128, "chunk size");
   static_assert(kTmemCols <= 512, "tensor memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -184,13 +191,14 @@ __device__ __forceinline__ float token_factor(const FfnParams& p, int row) {
   return p.rowscale != nullptr ? __ldg(p.rowscale + row) : 1.0f;
 }
 
-template <int NMAT, int BN, int WS, int BS, int AS, int DB>
+template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC>
 __global__ void __launch_bounds__(kThreads, 1)
 ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0,
                 const __grid_constant__ CUtensorMap tm_scales0, const __grid_constant__ CUtensorMap tm_codes1,
                 const __grid_constant__ CUtensorMap tm_scales1, const __grid_constant__ CUtensorMap tm_act) {
   pdl_enter();
-  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB>;
+  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB, KC>;
+  constexpr int kCPW = Cfg::kCPW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* w_smem = smem;
@@ -297,15 +305,16 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
           const int as = q % AS, bs = q % BS;
           const uint64_t bd = make_sdesc_sw128(smem_u32(b_smem + bs * Cfg::kBStageBytes));
           const uint32_t d0 = tmem + ds * NMAT * BN;
-          const uint32_t a0 = tmem + Cfg::kDCols + as * NMAT * 32;
+          const uint32_t a0 = tmem + Cfg::kDCols + as * NMAT * Cfg::kACols;
           const uint32_t acc0 = c > kc0 ? 1u : 0u;
 #pragma unroll
-          for (int m = 0; m < NMAT; ++m) mma_ts_f16(d0 + m * BN, a0 + m * 32, bd, idesc, acc0);
+          for (int m = 0; m < NMAT; ++m) mma_ts_f16(d0 + m * BN, a0 + m * Cfg::kACols, bd, idesc, acc0);
 #pragma unroll
-          for (int j = 1; j < kKC / 16; ++j)
+          for (int j = 1; j < KC / 16; ++j)
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m)   // K slice j: +32 bytes of B (+2 in the descriptor's address field)
-              mma_ts_f16_acc(d0 + m * BN, a0 + m * 32 + 8 * j, bd + uint64_t(2 * j), idesc);
+            for (int m = 0; m < NMAT; ++m)   // K slice j: atom j / 4 (+kBAtomBytes), +32 bytes per slice in it
+              mma_ts_f16_acc(d0 + m * BN, a0 + m * Cfg::kACols + 8 * j,
+                             bd + uint64_t((j / 4) * (Cfg::kBAtomBytes >> 4) + 2 * (j % 4)), idesc);
           mma_commit(&a_empty[as]);
           mma_commit(&b_empty[bs]);
         }
@@ -337,8 +346,11 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
         for (int c = kc0; c < kc1; ++c, ++q) {
           const int bs = q % BS;
           if (!(ok = ab.wait(&b_empty[bs], ((q / BS) & 1) ^ 1, kTagBEmpty, q, u))) break;
-          mbar_arrive_expect_tx(&b_full[bs], uint32_t(BN) * 128u);
-          tma_load_2d(b_smem + bs * Cfg::kBStageBytes, &tm_act, &b_full[bs], c * kKC, rb);
+          mbar_arrive_expect_tx(&b_full[bs], uint32_t(Cfg::kBStageBytes));
+#pragma unroll
+          for (int a = 0; a < Cfg::kAtoms; ++a)   // K past the end reads as zeros (their A is zero too)
+            tma_load_2d(b_smem + bs * Cfg::kBStageBytes + a * Cfg::kBAtomBytes, &tm_act, &b_full[bs],
+                        c * KC + a * kAtomK, rb);
         }
       }
       for (uint32_t j = (q > BS ? q - BS : 0); j < q; ++j) {   // drain
@@ -397,12 +409,16 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
           for (int m = 0; m < NMAT; ++m) {
             const uint8_t* base = w_smem + (s * NMAT + m) * kMatStageBytes;
             const uint8_t* crow = base + row * 128;
-            const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2 * cc) ^ (row & 7)) << 4));
-            const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2 * cc + 1) ^ (row & 7)) << 4));
-            const uint32_t sc = *reinterpret_cast<const uint32_t*>(base + kCodesBytes + row * 16 + cc * 4);
-            uint32_t o[32];
-            dequant_chunk(c0, c1, sc, o);
-            tmem_st_32x32b_x32(tmem + lane_base + Cfg::kDCols + (as * NMAT + m) * 32, o);
+#pragma unroll
+            for (int h = 0; h < Cfg::kAtoms; ++h) {   // 64 K of the chunk: 16-byte words 2t, 2t + 1, scale word t
+              const int t = cc * Cfg::kAtoms + h;
+              const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2 * t) ^ (row & 7)) << 4));
+              const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2 * t + 1) ^ (row & 7)) << 4));
+              const uint32_t sc = *reinterpret_cast<const uint32_t*>(base + kCodesBytes + row * 16 + t * 4);
+              uint32_t o[32];
+              dequant_chunk(c0, c1, sc, o);
+              tmem_st_32x32b_x32(tmem + lane_base + Cfg::kDCols + (as * NMAT + m) * Cfg::kACols + h * 32, o);
+            }
           }
           tmem_wait_st();
           tc_fence_before();

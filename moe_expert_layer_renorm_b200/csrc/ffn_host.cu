@@ -44,10 +44,11 @@ static int choose_splits(double units_est, int nkw, int num_sms, double split_co
 }
 
 // Prefill tile shapes <token rows (MMA N), weight stages, token stages, A
-// stages, accumulator buffers> of the two tcgen05 GEMMs.  Tensor memory
-// holds DB * NMAT * BN accumulator columns plus AS * NMAT * 32 for A.
-constexpr int kPreBN1 = 96, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 2, kPreDB1 = 2;
-constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 6, kPreAS2 = 4, kPreDB2 = 2;
+// stages, accumulator buffers, K per chunk> of the two tcgen05 GEMMs.
+// Tensor memory holds DB * NMAT * BN accumulator columns plus
+// AS * NMAT * KC / 2 for A.
+constexpr int kPreBN1 = 96, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 2, kPreDB1 = 2, kPreKC1 = 64;
+constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 3, kPreAS2 = 2, kPreDB2 = 2, kPreKC2 = 128;
 
 // Decode split-K: the smallest divisor of the K-stage count that gives every
 // SM a unit (a dynamic queue balances the rest, so waves do not matter).
@@ -79,8 +80,8 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
   pl.mt2 = (H + (pl.decode ? kDecRows : 128) - 1) / (pl.decode ? kDecRows : 128);
   pl.nkw1 = (H + kKW - 1) / kKW;
   pl.nkw2 = (I + kKW - 1) / kKW;
-  pl.nkc1 = H / kKC;
-  pl.nkc2 = I / kKC;
+  pl.nkc1 = (H + kPreKC1 - 1) / kPreKC1;
+  pl.nkc2 = (I + kPreKC2 - 1) / kPreKC2;
   if (pl.decode) {
     pl.g1 = {kDecBN, 1, 0, 4, 0, 0, 0};
     pl.g2 = {kDecBN, 1, 0, 4, 0, 0, 0};
@@ -185,13 +186,13 @@ static bool make_act_map(const void* base, int rows, int K, int box_rows, CUtens
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NMAT, int BN, int WS, int BS, int AS, int DB>
+template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC>
 static cudaError_t launch_gemm(const FfnParams& p, int grid, const CUtensorMap& c0, const CUtensorMap& s0,
                                const CUtensorMap& c1, const CUtensorMap& s1, const CUtensorMap& act,
                                cudaStream_t s) {
   ProfileScope prof(NMAT == 2 ? FT_KERNEL_GEMM_GATE_UP : FT_KERNEL_GEMM_DOWN, s);
-  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB>;
-  auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB>;
+  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB, KC>;
+  auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB, KC>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
@@ -318,9 +319,9 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
     const int grid = int(std::min<long long>(num_sms, pl.max_units1 + pl.max_units2));
     err = launch_decode(dp, grid, tmc, tms, tm_x, tm_h, s);
   } else {
-    err = launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    err = launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
     if (err == cudaSuccess)
-      err = launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
+      err = launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   }
   return err;
 }
