@@ -18,16 +18,35 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)T * vec_per_row) return;
   const int t = int(i / vec_per_row), c = int(i % vec_per_row);
+  const int32_t* rows = pair_to_row + size_t(t) * k;
+  const float* wt = w + size_t(t) * k;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < k; ++j) {
-    const int row = __ldg(pair_to_row + size_t(t) * k + j);
-    if (row < 0 || row >= P) { set_device_status(FT_DEV_BAD_INDEX); continue; }
-    const float wj = __ldg(w + size_t(t) * k + j);
-    const float4 o = __ldg(out_perm + size_t(row) * vec_per_row + c);
-    acc.x = fmaf(wj, o.x, acc.x);
-    acc.y = fmaf(wj, o.y, acc.y);
-    acc.z = fmaf(wj, o.z, acc.z);
-    acc.w = fmaf(wj, o.w, acc.w);
+  // eight selections at a time: their indices, weights and rows are all
+  // requested before the first is used (one memory round trip per batch
+  // instead of two per selection); the sum keeps the order j = 0 .. k-1
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    int row[8];
+    float wj[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      row[q] = j0 + q < k ? __ldg(rows + j0 + q) : -1;
+      wj[q] = j0 + q < k ? __ldg(wt + j0 + q) : 0.0f;
+    }
+    float4 o[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const bool ok = row[q] >= 0 && row[q] < P;
+      if (j0 + q < k && !ok) set_device_status(FT_DEV_BAD_INDEX);
+      o[q] = ok ? __ldg(out_perm + size_t(row[q]) * vec_per_row + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (row[q] < 0 || row[q] >= P) continue;   // also the padding past k (row -1)
+      acc.x = fmaf(wj[q], o[q].x, acc.x);
+      acc.y = fmaf(wj[q], o[q].y, acc.y);
+      acc.z = fmaf(wj[q], o[q].z, acc.z);
+      acc.w = fmaf(wj[q], o[q].w, acc.w);
+    }
   }
   y[size_t(t) * vec_per_row + c] = acc;
 }

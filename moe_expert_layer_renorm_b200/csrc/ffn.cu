@@ -657,29 +657,22 @@ __device__ void prep_schedule(const PrepParams& p, int b) {
   for (int i = first; i < p.ndone; i += stride) p.tile_done[i] = 0;
 }
 
-// One warp per permuted row r (token t = perm_src[r] / k): writes
-// x_perm[r] = f16(x[t] * 2^-s_t) and rowscale[r] = 2^s_t, with s_t >= 0 the
-// smallest shift that brings max|x[t]| below 2^15.  The f16 conversion is
-// then exact for every element of the row within a factor 2^32 of the row's
-// largest magnitude (bf16 has 8 significant bits, f16 subnormals reach
-// 2^-24); smaller elements round with an absolute error below 2^-41 max|x[t]|.
-// Rows in permuted order make each expert group's tokens one contiguous
-// block, so the GEMM loads them as plain tiles.
-__device__ void prep_rows(const PrepParams& p, int b) {
-  const int lane = threadIdx.x & 31;
-  const int r = b * (blockDim.x / 32) + threadIdx.x / 32;
-  if (r >= p.P) return;
-  const int t = __ldg(p.perm_src + r) / p.k_top;
-  const int nv = p.H / 8;
-  const uint4* row = p.x + size_t(t) * nv;
-  float m = 0.0f;
-  for (int c = lane; c < nv; c += 32) {
-    const uint4 v = __ldg(row + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+__device__ __forceinline__ float bf16x2_absmax(uint32_t w) {
+  return fmaxf(fabsf(__uint_as_float(w << 16)), fabsf(__uint_as_float(w & 0xFFFF0000u)));
+}
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& v, float f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
+  for (int q = 0; q < 4; ++q) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(w[q] << 16) * f, __uint_as_float(w[q] & 0xFFFF0000u) * f);
+    o[q] = *reinterpret_cast<const uint32_t*>(&h);
   }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The row's prescale shift from its largest magnitude (warp-wide max first).
+__device__ __forceinline__ int prep_shift(float m) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
   int shift = 0;
@@ -690,23 +683,62 @@ __device__ void prep_rows(const PrepParams& p, int b) {
   } else if (!(m <= 3.0e38f)) {
     set_device_status(FT_DEV_F16_RANGE);         // inf or nan input
   }
-  const float f = ldexpf(1.0f, -shift);
-  if (lane == 0) p.rowscale[r] = ldexpf(1.0f, shift);
-  uint4* out = p.x_perm + size_t(r) * nv;
-  for (int c = lane; c < nv; c += 32) {
-    const uint4 v = __ldg(row + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __half2 h = __floats2half2_rn(__uint_as_float(w[q] << 16) * f, __uint_as_float(w[q] & 0xFFFF0000u) * f);
-      o[q] = *reinterpret_cast<const uint32_t*>(&h);
-    }
-    out[c] = make_uint4(o[0], o[1], o[2], o[3]);
-  }
+  return shift;
 }
 
-__global__ void __launch_bounds__(256) ffn_prep_kernel(const PrepParams p) {
+// One warp per permuted row r (token t = perm_src[r] / k): writes
+// x_perm[r] = f16(x[t] * 2^-s_t) and rowscale[r] = 2^s_t, with s_t >= 0 the
+// smallest shift that brings max|x[t]| below 2^15.  The f16 conversion is
+// then exact for every element of the row within a factor 2^32 of the row's
+// largest magnitude (bf16 has 8 significant bits, f16 subnormals reach
+// 2^-24); smaller elements round with an absolute error below 2^-41 max|x[t]|.
+// Rows in permuted order make each expert group's tokens one contiguous
+// block, so the GEMM loads them as plain tiles.  Rows of up to 3072 values
+// are read once into registers with all loads in flight together (the
+// kernel is latency-bound at decode sizes); longer rows are read twice.
+__device__ void prep_rows(const PrepParams& p, int b) {
+  constexpr int kRegVec = 12;                    // 16-byte vectors per lane kept in registers
+  const int lane = threadIdx.x & 31;
+  const int r = b * (blockDim.x / 32) + threadIdx.x / 32;
+  if (r >= p.P) return;
+  const int t = __ldg(p.perm_src + r) / p.k_top;
+  const int nv = p.H / 8;
+  const uint4* row = p.x + size_t(t) * nv;
+  uint4* out = p.x_perm + size_t(r) * nv;
+  if (nv <= 32 * kRegVec) {
+    uint4 v[kRegVec];
+#pragma unroll
+    for (int i = 0; i < kRegVec; ++i) {
+      const int c = lane + 32 * i;
+      v[i] = c < nv ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kRegVec; ++i)
+      m = fmaxf(m, fmaxf(fmaxf(bf16x2_absmax(v[i].x), bf16x2_absmax(v[i].y)),
+                         fmaxf(bf16x2_absmax(v[i].z), bf16x2_absmax(v[i].w))));
+    const int shift = prep_shift(m);
+    const float f = ldexpf(1.0f, -shift);
+    if (lane == 0) p.rowscale[r] = ldexpf(1.0f, shift);
+#pragma unroll
+    for (int i = 0; i < kRegVec; ++i) {
+      const int c = lane + 32 * i;
+      if (c < nv) out[c] = bf16x8_to_f16x8(v[i], f);
+    }
+    return;
+  }
+  float m = 0.0f;
+  for (int c = lane; c < nv; c += 32) {
+    const uint4 v = __ldg(row + c);
+    m = fmaxf(m, fmaxf(fmaxf(bf16x2_absmax(v.x), bf16x2_absmax(v.y)), fmaxf(bf16x2_absmax(v.z), bf16x2_absmax(v.w))));
+  }
+  const int shift = prep_shift(m);
+  const float f = ldexpf(1.0f, -shift);
+  if (lane == 0) p.rowscale[r] = ldexpf(1.0f, shift);
+  for (int c = lane; c < nv; c += 32) out[c] = bf16x8_to_f16x8(__ldg(row + c), f);
+}
+
+__global__ void __launch_bounds__(256, 2) ffn_prep_kernel(const PrepParams p) {
   pdl_enter();
   if (int(blockIdx.x) < p.nsched) prep_schedule(p, blockIdx.x);
   else prep_rows(p, blockIdx.x - p.nsched);
