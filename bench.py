@@ -19,6 +19,7 @@ import hashlib
 import io
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -119,15 +120,23 @@ class ClockSampler:
 
 # ------------------------------------------------------------ our arm ---
 
+def _code_only(text: str) -> str:
+    """C++/CUDA source with comments and blank lines removed (the kernels'
+    sources contain no string literal holding a comment marker)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash() -> str:
-    """Hash of the sources of the two expert GEMM kernels, the helpers they
-    include and the host code that sizes their launches: a counter taken on
-    other sources no longer describes the launches that run."""
+    """Hash of the code (comments excluded) of the expert FFN kernels, the
+    helpers they include and the host code that sizes their launches: a
+    counter taken on other code no longer describes the launches that run."""
     d = os.path.join(ROOT, "moe_expert_layer_renorm_b200", "csrc")
     h = hashlib.sha256()
     for name in ("sm100.cuh", "ffn.cu", "decode.cu", "ffn_host.cu"):
-        with open(os.path.join(d, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(d, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

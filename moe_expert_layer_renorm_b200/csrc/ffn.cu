@@ -5,23 +5,26 @@
 // rows of that expert's group, so any group size from 1 row up maps onto one
 // instruction shape (N = group rows rounded up to 16).
 //
-// Data path of one CTA (persistent; 16 warps):
+// Data path of one CTA (persistent; 16 warps), per KC-wide chunk of K:
 //   warp 0      TMA: packed E2M1 codes (128 rows x 128 B, 128-byte swizzle)
 //               and E4M3 scales (128 rows x 16 B) of each matrix, 256 K per stage
-//   warp 2      TMA: the unit's token rows (f16, 64 K per chunk) into
-//               128-byte-swizzled K-major shared memory (the MMA's B operand),
-//               16-row tiles of the permuted f16 activations (GEMM1) or of h
+//   warp 2      TMA: the unit's token rows (f16) into 128-byte-swizzled K-major
+//               shared memory (the MMA's B operand): one BN-row box per 64-K
+//               swizzle atom, of the permuted f16 activations (GEMM1) or of h
 //               (GEMM2); both are stored in permuted row order
-//   warps 4-11  dequantise one 64-K chunk per step: E2M1 -> f16 (cvt) times the
-//               E4M3 block scale (exact in f16), widened to bf16 (exact), and
-//               stored with tcgen05.st straight into tensor memory, where the
-//               MMA reads it as its A operand (no shared-memory round trip)
-//   warp 3      idle
-//   warp 1      one thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
-//               accumulators in tensor memory) and commits to the barriers
+//   warps 4-11  two warpgroups, alternate chunks: E2M1 -> f16 (cvt) times the
+//               E4M3 block scale (exact in f16), stored with tcgen05.st
+//               straight into tensor memory, where the MMA reads it as its A
+//               operand (no shared-memory round trip)
+//   warp 3      waits on the operand barriers for the MMA warp and hands each
+//               ready chunk over at a named barrier
+//   warp 1      one thread issues tcgen05.mma kind::f16 (f16 x f16 -> fp32
+//               accumulators in tensor memory) and commits to the barriers;
+//               it waits on no mbarrier inside its loop
 //   warps 12-15 epilogue: tcgen05.ld of the accumulators, fp32 global scale,
-//               SwiGLU (GEMM1) and bf16 stores; for split-K, fp32 partials and
-//               a last-arriving-CTA reduction in a fixed order (deterministic)
+//               SwiGLU (GEMM1) and f16 h / fp32 output stores; for split-K,
+//               fp32 partials and a last-arriving-CTA reduction in a fixed
+//               order (deterministic)
 //
 // Every pipeline wait is bounded (see sm100.cuh); a wait that gives up sets
 // the device status word and an abort flag, all roles leave their loops, and

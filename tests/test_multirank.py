@@ -79,3 +79,15 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "tokens/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    """The traffic records are keyed by the kernels' code: a comment edit keeps
+    the key, a code edit changes it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    src = "// header\nint f(int x) {  // trailing\n  /* block\n comment */ return x + 1;\n}\n\n"
+    assert bench._code_only(src) == bench._code_only(src.replace("trailing", "other words"))
+    assert bench._code_only(src) != bench._code_only(src.replace("x + 1", "x + 2"))
+    assert "header" not in bench._code_only(src) and "block" not in bench._code_only(src)
+    assert len(bench.kernel_source_hash()) == 16
