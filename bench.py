@@ -48,6 +48,8 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--slot-churn", action="store_true",
+                    help="measure the expert-cache miss path (pinned host banks, LRU slot manager) instead")
     return ap.parse_args()
 
 
@@ -527,10 +529,44 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+CHURN_CONFIG = dict(T=8, E=128, k=8, H=2048, I=768, layers=8, domains=4, hot=16, capacity=192)
+
+
+def run_slot_churn(args):
+    """Expert-cache churn (one GPU): decode steps of 8 layers (E128 k8 H2048
+    I768, T=8) whose experts live in pinned host banks; the device pool holds
+    192 slots, 1.5 domains' worth.  The domain switches every
+    `steps_per_domain` steps, so the first step of a domain misses on every
+    layer.  Both work orders (demand, prefetch) are timed with CUDA events."""
+    import torch
+    from moe_expert_layer_renorm_b200 import churn
+
+    cfg = churn.ChurnConfig(**CHURN_CONFIG)
+    hs = churn.hot_sets(cfg)
+    banks = churn.ExpertBanks(cfg, hs)
+    out = {"metric": "expert-cache churn: decode step time with misses (switch) and without (steady)",
+           "unit": "ms/step", "n_gpus": 1, "data": "synthetic (domain-rotation routing)",
+           "config": dict(CHURN_CONFIG, steps_per_domain=8, rounds=2, slot_mb=round(banks.slot_bytes / 1e6, 3))}
+    for mode in ("demand", "prefetch"):
+        r = churn.run_churn(cfg, mode, steps_per_domain=8, rounds=2, banks=banks)
+        sw, st = statistics.median(r["switch_ms"]), statistics.median(r["steady_ms"])
+        miss = statistics.median(r["misses_per_switch"])
+        bytes_sw = statistics.median(r["h2d_bytes_per_switch"])
+        out[mode] = {"switch_ms": round(sw, 4), "steady_ms": round(st, 4), "misses_per_switch": miss,
+                     "h2d_MB_per_switch": round(bytes_sw / 1e6, 1),
+                     "miss_cost_ms": round(sw - st, 4),
+                     "h2d_GBps_effective": round(bytes_sw / max(sw - st, 1e-6) / 1e6, 1),
+                     "stats": r["stats"]}
+        torch.cuda.synchronize()
+    print(json.dumps(out))
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.slot_churn:
+        run_slot_churn(args)
     else:
         run_ours(args)
 

@@ -9,7 +9,12 @@
 //      most-recently-used end and is pinned for this call;
 //   2. every miss takes a free slot, else evicts the least recently used
 //      slot not pinned by this call, and is filled from its pinned host bank
-//      with one cudaMemcpyAsync on the copy stream;
+//      with one cudaMemcpyAsync on the copy stream.  A fill that reuses a
+//      slot waits on the copy stream only for the compute work that last
+//      used that slot: each acquire records an event on the compute stream
+//      (everything enqueued so far), which becomes the last-use mark of the
+//      slots the previous acquire handed out.  So fills for the next layer
+//      overlap the current layer's kernels unless they evict its slots;
 //   3. the device slot table [E] is uploaded on the copy stream, an event is
 //      recorded there and the compute stream waits on it.
 // More distinct experts than capacity -> FT_ERR_CAPACITY (nothing changes).
@@ -45,7 +50,14 @@ struct ft_slot_mgr {
   int32_t* pinned_table = nullptr;      // page-locked staging for the async upload
   int pinned_table_len = 0;
   cudaEvent_t done = nullptr;
-  cudaEvent_t compute_mark = nullptr;   // compute-stream position when a fill evicts a slot
+  // last-use marks: a ring of events recorded on the compute stream, one per
+  // acquire; slot_mark[s] indexes the ring (-1: never used).  A ring entry may
+  // be re-recorded later than the use it marks, which only makes a wait longer.
+  static constexpr int kMarks = 64;
+  cudaEvent_t marks[kMarks] = {};
+  int next_mark = 0;
+  std::vector<int> slot_mark;
+  std::vector<int> prev_slots;          // slots handed out by the previous acquire
   ft_slot_stats_t stats{};
   int inject_failures = 0;
   bool host_only = false;               // FT_SLOT_HOST_ONLY: bookkeeping only, no CUDA calls
@@ -69,10 +81,16 @@ extern "C" int ft_slot_create(ft_slot_mgr** mgr, int capacity, const ft_nvfp4_sl
   m->pool = static_cast<uint8_t*>(device_pool);
   m->host_only = host_only;
   for (int s = capacity - 1; s >= 0; --s) m->free_slots.push_back(s);
-  if (!host_only && (cudaEventCreateWithFlags(&m->done, cudaEventDisableTiming) != cudaSuccess ||
-                     cudaEventCreateWithFlags(&m->compute_mark, cudaEventDisableTiming) != cudaSuccess)) {
+  m->slot_mark.assign(capacity, -1);
+  bool ok = true;
+  if (!host_only) {
+    ok = cudaEventCreateWithFlags(&m->done, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < ft_slot_mgr::kMarks && ok; ++i)
+      ok = cudaEventCreateWithFlags(&m->marks[i], cudaEventDisableTiming) == cudaSuccess;
+  }
+  if (!ok) {
     ftmoe::set_last_error("ft_slot_create: cudaEventCreate failed");
-    delete m;
+    ft_slot_destroy(m);
     return FT_ERR_CUDA;
   }
   *mgr = m;
@@ -128,6 +146,18 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
       return FT_ERR_NOT_RESIDENT;
     }
   }
+  // the work enqueued on the compute stream so far is the last use of the
+  // slots the previous acquire handed out
+  if (!m->host_only && !m->prev_slots.empty()) {
+    const int mk = m->next_mark;
+    if (cudaEventRecord(m->marks[mk], reinterpret_cast<cudaStream_t>(compute)) != cudaSuccess) {
+      ftmoe::set_last_error("ft_slot_acquire: recording the compute mark failed");
+      return FT_ERR_CUDA;
+    }
+    m->next_mark = (mk + 1) % ft_slot_mgr::kMarks;
+    for (int sl : m->prev_slots) m->slot_mark[sl] = mk;
+    m->prev_slots.clear();
+  }
   // pin: hits move to the front; they are protected from eviction by this call
   std::unordered_map<uint64_t, char> pinned;
   for (int e : want) {
@@ -141,9 +171,6 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
   }
   std::vector<int32_t> table(table_len, -1);
   const size_t slot_bytes = size_t(m->layout.slot_bytes);
-  // A slot may still be read by work already enqueued on the compute stream:
-  // fills that reuse an evicted slot wait for that work on the copy stream.
-  bool copy_waits = false;
   for (int e : want) {
     const uint64_t key = slot_key(layer, e);
     auto it = m->resident.find(key);
@@ -168,15 +195,14 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
       m->resident.erase(*victim);
       m->lru.erase(victim);
       ++m->stats.evictions;
-      if (!m->host_only && !copy_waits) {
-        if (cudaEventRecord(m->compute_mark, reinterpret_cast<cudaStream_t>(compute)) != cudaSuccess ||
-            cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(copy), m->compute_mark, 0) != cudaSuccess) {
-          m->free_slots.push_back(slot);
-          ftmoe::set_last_error("ft_slot_acquire: ordering the fill after compute failed");
-          return FT_ERR_CUDA;
-        }
-        copy_waits = true;
-      }
+    }
+    // the slot may still be read by compute work enqueued before: the fill
+    // waits for the last use of this slot on the copy stream
+    if (!m->host_only && m->slot_mark[slot] >= 0 &&
+        cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(copy), m->marks[m->slot_mark[slot]], 0) != cudaSuccess) {
+      m->free_slots.push_back(slot);
+      ftmoe::set_last_error("ft_slot_acquire: ordering the fill after compute failed");
+      return FT_ERR_CUDA;
     }
     cudaError_t err = cudaSuccess;
     if (m->inject_failures > 0) {
@@ -198,6 +224,7 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
     m->stats.bytes_h2d += int64_t(slot_bytes);
   }
   m->host_table = table;
+  for (int e : want) m->prev_slots.push_back(table[e]);
   if (m->host_only) {   // device_table is host memory in this mode
     std::memcpy(device_table, table.data(), size_t(table_len) * 4);
     return FT_OK;
@@ -243,7 +270,8 @@ extern "C" int ft_slot_destroy(ft_slot_mgr* m) {
     cudaEventSynchronize(m->done);
     cudaEventDestroy(m->done);
   }
-  if (m->compute_mark) cudaEventDestroy(m->compute_mark);
+  for (cudaEvent_t ev : m->marks)
+    if (ev) cudaEventDestroy(ev);
   if (m->pinned_table) cudaFreeHost(m->pinned_table);
   delete m;
   return FT_OK;
