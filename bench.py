@@ -48,8 +48,9 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--slot-churn", action="store_true",
-                    help="measure the expert-cache miss path (pinned host banks, LRU slot manager) instead")
+    ap.add_argument("--slot-churn", nargs="?", const="decode", default=None, choices=["decode", "prefill_stream"],
+                    help="measure the expert-cache miss path (pinned host banks, LRU slot manager) instead: "
+                         "domain-rotation decode steps, or prefill layers streamed through a two-layer pool")
     return ap.parse_args()
 
 
@@ -541,6 +542,9 @@ def run_slot_churn(args):
     import torch
     from moe_expert_layer_renorm_b200 import churn
 
+    if args.slot_churn == "prefill_stream":
+        run_prefill_stream()
+        return
     cfg = churn.ChurnConfig(**CHURN_CONFIG)
     hs = churn.hot_sets(cfg)
     banks = churn.ExpertBanks(cfg, hs)
@@ -559,6 +563,35 @@ def run_slot_churn(args):
                      "stats": r["stats"]}
         torch.cuda.synchronize()
     print(json.dumps(out))
+
+
+STREAM_CONFIG = dict(T=4096, E=128, k=8, H=2048, I=768, layers=4, domains=1, hot=128, capacity=256)
+
+
+def run_prefill_stream():
+    """Double-buffered prefill expert streaming (one GPU): 4 prefill layers
+    (T=4096, E128 k8 H2048 I768, uniform routing) whose 128 experts each come
+    from pinned host banks into a 256-slot pool (two layers' worth): layer
+    l + 1's experts are filled while layer l runs.  Reports the streamed step,
+    the same step with every expert resident, and a plain copy of the same
+    bytes."""
+    import torch
+    from moe_expert_layer_renorm_b200 import churn
+
+    cfg = churn.ChurnConfig(**STREAM_CONFIG)
+    banks = churn.ExpertBanks(cfg, churn.hot_sets(cfg), keep_device=True)
+    r = churn.run_stream(cfg, steps=4, banks=banks)
+    sm, rm = statistics.median(r["stream_ms"]), statistics.median(r["resident_ms"])
+    b = statistics.median(r["h2d_bytes_per_step"])
+    copy_ms = b / (r["copy_only_GBps"] * 1e6)
+    print(json.dumps({
+        "metric": "prefill expert streaming: step time of 4 layers with every expert filled from the host",
+        "unit": "ms/step", "n_gpus": 1, "data": "synthetic (uniform routing)",
+        "config": dict(STREAM_CONFIG, steps=4, slot_mb=round(banks.slot_bytes / 1e6, 3)),
+        "stream_ms": round(sm, 3), "resident_ms": round(rm, 3), "h2d_MB_per_step": round(b / 1e6, 1),
+        "copy_only_GBps": round(r["copy_only_GBps"], 1), "copy_only_ms_for_step_bytes": round(copy_ms, 3),
+        "overlap": round((rm + copy_ms - sm) / min(rm, copy_ms), 3),
+        "stats": r["stats"]}))
 
 
 def main():

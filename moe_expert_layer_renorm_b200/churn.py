@@ -197,4 +197,50 @@ def run_churn(cfg: ChurnConfig, mode: str, steps_per_domain: int, rounds: int, b
             "h2d_bytes_per_switch": h2d, "stats": st}
 
 
-__all__ = ["ChurnConfig", "ExpertBanks", "ChurnRun", "hot_sets", "step_logits", "run_churn"]
+def run_stream(cfg: ChurnConfig, steps: int, banks: ExpertBanks, device="cuda") -> dict:
+    """Streaming: every layer of every step needs experts that are not on the
+    device (a pool of two layers' worth shared by `layers` > 2 layers), so
+    each layer's experts are filled while the previous layer runs (prefetch
+    order, a double-buffered pool).  Also times the same steps with every
+    expert resident (banks.resident) and the fills alone."""
+    assert banks.resident is not None
+    hs = hot_sets(cfg)
+    run = ChurnRun(cfg, banks, device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream_ms, resident_ms, h2d = [], [], []
+    tables = [banks.resident_table(cfg, l) for l in range(cfg.layers)]
+    for step in range(steps + 1):
+        logits = [torch.from_numpy(step_logits(cfg, hs, l, 0, step)).to(device) for l in range(cfg.layers)]
+        torch.cuda.synchronize()
+        before = run.mgr.stats()
+        ev0.record(run.compute)
+        run.step(logits, "prefetch")
+        ev1.record(run.compute)
+        torch.cuda.synchronize()
+        after = run.mgr.stats()
+        if step > 0:
+            stream_ms.append(ev0.elapsed_time(ev1))
+            h2d.append(after["bytes_h2d"] - before["bytes_h2d"])
+        ev0.record(run.compute)
+        for l in range(cfg.layers):
+            run.layers[l].forward(run.x[l], logits[l], tables[l], banks.resident, run.compute)
+        ev1.record(run.compute)
+        torch.cuda.synchronize()
+        if step > 0:
+            resident_ms.append(ev0.elapsed_time(ev1))
+    # the fills alone: the same bytes as one step, slot images from the banks
+    n = min(cfg.capacity, banks.host.shape[0])
+    with torch.cuda.stream(run.copy):
+        ev0.record(run.copy)
+        for i in range(n):
+            run.pool.slot_view(i).copy_(banks.host[i], non_blocking=True)
+        ev1.record(run.copy)
+    torch.cuda.synchronize()
+    copy_gbps = n * banks.slot_bytes / (ev0.elapsed_time(ev1) * 1e6)
+    st = run.mgr.stats()
+    run.mgr.close()
+    return {"stream_ms": stream_ms, "resident_ms": resident_ms, "h2d_bytes_per_step": h2d,
+            "copy_only_GBps": copy_gbps, "stats": st}
+
+
+__all__ = ["ChurnConfig", "ExpertBanks", "ChurnRun", "hot_sets", "step_logits", "run_churn", "run_stream"]

@@ -47,9 +47,15 @@ struct ft_slot_mgr {
   std::unordered_map<uint64_t, const void*> banks;
   std::vector<int> free_slots;
   std::vector<int32_t> host_table;      // staging copy of the last uploaded table
-  int32_t* pinned_table = nullptr;      // page-locked staging for the async upload
+  // page-locked staging of the table uploads: a ring, so that an acquire
+  // blocks the host only when the upload of kStage calls ago is still
+  // pending (with one buffer, every acquire waited for the previous call's
+  // fills, which left the copy engine idle while the host queued the next)
+  static constexpr int kStage = 8;
+  int32_t* pinned_table[kStage] = {};
+  cudaEvent_t staged[kStage] = {};     // upload of pinned_table[i] (and the fills before it) done
   int pinned_table_len = 0;
-  cudaEvent_t done = nullptr;
+  int next_stage = 0;
   // last-use marks: a ring of events recorded on the compute stream, one per
   // acquire; slot_mark[s] indexes the ring (-1: never used).  A ring entry may
   // be re-recorded later than the use it marks, which only makes a wait longer.
@@ -84,7 +90,8 @@ extern "C" int ft_slot_create(ft_slot_mgr** mgr, int capacity, const ft_nvfp4_sl
   m->slot_mark.assign(capacity, -1);
   bool ok = true;
   if (!host_only) {
-    ok = cudaEventCreateWithFlags(&m->done, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < ft_slot_mgr::kStage && ok; ++i)
+      ok = cudaEventCreateWithFlags(&m->staged[i], cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; i < ft_slot_mgr::kMarks && ok; ++i)
       ok = cudaEventCreateWithFlags(&m->marks[i], cudaEventDisableTiming) == cudaSuccess;
   }
@@ -171,6 +178,7 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
   }
   std::vector<int32_t> table(table_len, -1);
   const size_t slot_bytes = size_t(m->layout.slot_bytes);
+  std::vector<char> waited(ft_slot_mgr::kMarks, 0);   // one stream wait per distinct mark
   for (int e : want) {
     const uint64_t key = slot_key(layer, e);
     auto it = m->resident.find(key);
@@ -198,11 +206,14 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
     }
     // the slot may still be read by compute work enqueued before: the fill
     // waits for the last use of this slot on the copy stream
-    if (!m->host_only && m->slot_mark[slot] >= 0 &&
-        cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(copy), m->marks[m->slot_mark[slot]], 0) != cudaSuccess) {
-      m->free_slots.push_back(slot);
-      ftmoe::set_last_error("ft_slot_acquire: ordering the fill after compute failed");
-      return FT_ERR_CUDA;
+    const int mk = m->slot_mark[slot];
+    if (!m->host_only && mk >= 0 && !waited[mk]) {
+      if (cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(copy), m->marks[mk], 0) != cudaSuccess) {
+        m->free_slots.push_back(slot);
+        ftmoe::set_last_error("ft_slot_acquire: ordering the fill after compute failed");
+        return FT_ERR_CUDA;
+      }
+      waited[mk] = 1;
     }
     cudaError_t err = cudaSuccess;
     if (m->inject_failures > 0) {
@@ -231,27 +242,30 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
   }
   // upload the table from page-locked staging so the copy stays asynchronous
   if (m->pinned_table_len < table_len) {
-    // the previous upload (if any) must have finished reading the old buffer
-    if (m->pinned_table) {
-      cudaEventSynchronize(m->done);
-      cudaFreeHost(m->pinned_table);
+    // every pending upload must have finished reading the old buffers
+    for (int i = 0; i < ft_slot_mgr::kStage; ++i) {
+      cudaEventSynchronize(m->staged[i]);
+      if (m->pinned_table[i]) cudaFreeHost(m->pinned_table[i]);
+      m->pinned_table[i] = nullptr;
     }
-    m->pinned_table = nullptr;
     m->pinned_table_len = 0;
-    if (cudaMallocHost(reinterpret_cast<void**>(&m->pinned_table), size_t(table_len) * 4) != cudaSuccess) {
-      ftmoe::set_last_error("ft_slot_acquire: cudaMallocHost failed");
-      return FT_ERR_CUDA;
+    for (int i = 0; i < ft_slot_mgr::kStage; ++i) {
+      if (cudaMallocHost(reinterpret_cast<void**>(&m->pinned_table[i]), size_t(table_len) * 4) != cudaSuccess) {
+        ftmoe::set_last_error("ft_slot_acquire: cudaMallocHost failed");
+        return FT_ERR_CUDA;
+      }
     }
     m->pinned_table_len = table_len;
-  } else {
-    cudaEventSynchronize(m->done);  // previous upload finished reading the staging buffer
   }
-  std::memcpy(m->pinned_table, table.data(), size_t(table_len) * 4);
+  const int st = m->next_stage;
+  m->next_stage = (st + 1) % ft_slot_mgr::kStage;
+  cudaEventSynchronize(m->staged[st]);   // the upload kStage calls ago finished reading this buffer
+  std::memcpy(m->pinned_table[st], table.data(), size_t(table_len) * 4);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy);
-  if (cudaMemcpyAsync(device_table, m->pinned_table, size_t(table_len) * 4, cudaMemcpyHostToDevice, cs) !=
+  if (cudaMemcpyAsync(device_table, m->pinned_table[st], size_t(table_len) * 4, cudaMemcpyHostToDevice, cs) !=
           cudaSuccess ||
-      cudaEventRecord(m->done, cs) != cudaSuccess ||
-      cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(compute), m->done, 0) != cudaSuccess) {
+      cudaEventRecord(m->staged[st], cs) != cudaSuccess ||
+      cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(compute), m->staged[st], 0) != cudaSuccess) {
     ftmoe::set_last_error("ft_slot_acquire: table upload failed");
     return FT_ERR_CUDA;
   }
@@ -266,13 +280,15 @@ extern "C" int ft_slot_stats(const ft_slot_mgr* m, ft_slot_stats_t* out) {
 
 extern "C" int ft_slot_destroy(ft_slot_mgr* m) {
   if (!m) return FT_ERR_INVALID_ARG;
-  if (m->done) {
-    cudaEventSynchronize(m->done);
-    cudaEventDestroy(m->done);
+  for (int i = 0; i < ft_slot_mgr::kStage; ++i) {
+    if (m->staged[i]) {
+      cudaEventSynchronize(m->staged[i]);
+      cudaEventDestroy(m->staged[i]);
+    }
+    if (m->pinned_table[i]) cudaFreeHost(m->pinned_table[i]);
   }
   for (cudaEvent_t ev : m->marks)
     if (ev) cudaEventDestroy(ev);
-  if (m->pinned_table) cudaFreeHost(m->pinned_table);
   delete m;
   return FT_OK;
 }
