@@ -268,8 +268,15 @@ FT_API int ft_slot_register_host(ft_slot_mgr* mgr, int layer, int expert, const 
  * until the next acquire; misses evict the least recently used unpinned
  * slots.  Returns FT_ERR_CAPACITY when more distinct experts are requested
  * than the pool can hold, FT_ERR_NOT_RESIDENT when a miss has no host bank.
- * Synchronous on the host; the table upload and fills are enqueued on `copy`
- * and `compute` waits for them.
+ * The bookkeeping is synchronous on the host; the fills and the table upload
+ * are enqueued on `copy` and `compute` waits for them.  A fill that reuses a
+ * slot first waits (on `copy`) for the compute work that last read that slot:
+ * the work enqueued on `compute` before the acquire that followed the one
+ * which handed the slot out.  So the fills of the next layer overlap the
+ * current layer's kernels.  The host blocks only when the table upload of
+ * eight calls earlier is still pending (a ring of page-locked staging
+ * buffers).  device_slot_table must not be read by kernels still in flight
+ * when it is passed again: use one table per layer in flight.
  */
 FT_API int ft_slot_acquire(ft_slot_mgr* mgr, int layer, const int32_t* host_expert_ids, int n,
                     int32_t* device_slot_table, int table_len, ft_stream_t compute, ft_stream_t copy);
