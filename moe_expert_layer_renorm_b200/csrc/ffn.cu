@@ -335,7 +335,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
     }
   } else if (warp == 2) {
     // --------------------------------------------- B (token) producer ---
-    // Lane 0 issues one BN-row TMA box per 64-K chunk (one large box keeps
+    // Lane 0 issues one BN-row TMA box per 64-K swizzle atom (one large box keeps
     // the copy engine's per-box cost off the critical path; 16-row boxes
     // were several times slower).  Rows past the group end are other
     // groups' rows (or zero fill past the last row): finite, and their
