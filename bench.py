@@ -199,6 +199,59 @@ def workload_config(w, R: int, S: int, world: int, distinct: float) -> dict:
                   % (R, step_mb, (R - 1) * step_mb)}
 
 
+class E2EPipeline:
+    """End-to-end steps with host buffers, overlapped across steps.
+
+    nbuf buffer sets (device inputs, layer buffers, host result) alternate
+    between steps.  Step i's inputs are copied in on the h2d stream while step
+    i - 1 computes, and its result is copied out on the d2h stream while step
+    i + 1 computes.  Every step still copies its own inputs in and its own
+    result out.  Ordering (all by events, nothing on the host):
+      copy_in(i)   waits until replay(i - nbuf) has read buffer i % nbuf;
+      replay(i)    waits for copy_in(i) and for copy_out(i - nbuf), which
+                   must have read the layer output that replay(i) overwrites;
+      copy_out(i)  waits for replay(i).
+    copy_in, replay and copy_out are callables (step, buffer, stream)."""
+
+    def __init__(self, nbuf, h2d, compute, d2h, make_event, copy_in, replay, copy_out):
+        self.nbuf, self.h2d, self.compute, self.d2h = nbuf, h2d, compute, d2h
+        self.copy_in, self.replay, self.copy_out = copy_in, replay, copy_out
+        self.in_ready = [make_event() for _ in range(nbuf)]
+        self.computed = [make_event() for _ in range(nbuf)]
+        self.out_done = [make_event() for _ in range(nbuf)]
+
+    def _in(self, i):
+        b = i % self.nbuf
+        self.h2d.wait_event(self.computed[b])
+        self.copy_in(i, b, self.h2d)
+        self.in_ready[b].record(self.h2d)
+
+    def _compute_out(self, i):
+        b = i % self.nbuf
+        self.compute.wait_event(self.in_ready[b])
+        self.compute.wait_event(self.out_done[b])
+        self.replay(i, b, self.compute)
+        self.computed[b].record(self.compute)
+        self.d2h.wait_event(self.computed[b])
+        self.copy_out(i, b, self.d2h)
+        self.out_done[b].record(self.d2h)
+
+    def run(self, n, start_event=None):
+        """Enqueue n steps; the compute stream ends after the last copy-out.
+        start_event (recorded on the compute stream) gates the copy streams."""
+        if start_event is not None:
+            self.h2d.wait_event(start_event)
+            self.d2h.wait_event(start_event)
+        if n <= 0:
+            return
+        self._in(0)
+        for i in range(n):
+            if i + 1 < n:
+                self._in(i + 1)
+            self._compute_out(i)
+        self.compute.wait_event(self.out_done[(n - 1) % self.nbuf])
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -305,30 +358,73 @@ def run_ours(args):
     host = []
     for L in layers:
         host.append((L["x"].cpu().pin_memory(), L["lg"].cpu().pin_memory()))
-    y_host = torch.empty((T, w.H), dtype=torch.float32).pin_memory()
-    xd = torch.empty_like(layers[0]["x"])
-    lgd = torch.empty_like(layers[0]["lg"])
-    e2e_graphs = []
-    for l in range(R):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(g, stream=stream):
-                layer.forward(xd, lgd, layers[l]["st"], layers[l]["pool"], stream=stream)
-        e2e_graphs.append(g)
+    bufs = []
+    for _ in range(2):
+        bufs.append(dict(lay=MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev),
+                         xd=torch.empty_like(layers[0]["x"]), lgd=torch.empty_like(layers[0]["lg"]),
+                         y_host=torch.empty((T, w.H), dtype=torch.float32).pin_memory()))
+    e2e_graphs = {}
+    for bi, B in enumerate(bufs):
+        for l in range(R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    B["lay"].forward(B["xd"], B["lgd"], layers[l]["st"], layers[l]["pool"], stream=stream)
+            e2e_graphs[(l, bi)] = g
+    h2d_stream = torch.cuda.Stream(device=dev)
+    d2h_stream = torch.cuda.Stream(device=dev)
 
-    def e2e_step(i):
+    def e2e_in(i, bi, s):
         hx, hl = host[i % R]
-        xd.copy_(hx, non_blocking=True)
-        lgd.copy_(hl, non_blocking=True)
-        e2e_graphs[i % R].replay()
-        y_host.copy_(layer.y, non_blocking=True)
+        with torch.cuda.stream(s):
+            bufs[bi]["xd"].copy_(hx, non_blocking=True)
+            bufs[bi]["lgd"].copy_(hl, non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        for i in range(3):
-            e2e_step(i)
-    stream.synchronize()
-    e2e_ms = timed(e2e_step, args.steps)
-    for g in graphs + e2e_graphs:
+    def e2e_replay(i, bi, s):
+        with torch.cuda.stream(s):
+            e2e_graphs[(i % R, bi)].replay()
+
+    def e2e_out(i, bi, s):
+        with torch.cuda.stream(s):
+            bufs[bi]["y_host"].copy_(bufs[bi]["lay"].y, non_blocking=True)
+
+    pipe = E2EPipeline(2, h2d_stream, stream, d2h_stream, torch.cuda.Event, e2e_in, e2e_replay, e2e_out)
+
+    def timed_e2e(n):
+        """Like timed(): CUDA-event time of n pipelined end-to-end steps, max over ranks."""
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(2_000_000)
+            a.record(stream)
+        pipe.run(n, start_event=a)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b), dev)
+
+    def serial_e2e_step(i):
+        """One step with its copies on the compute stream, nothing overlapped."""
+        e2e_in(i, 0, stream)
+        e2e_replay(i, 0, stream)
+        e2e_out(i, 0, stream)
+
+    e2e_pipelined, e2e_note = True, None
+    try:
+        pipe.run(3)
+        torch.cuda.synchronize()
+        e2e_ms = timed_e2e(args.steps)
+    except (RuntimeError, TypeError, AttributeError) as exc:   # report it, and measure the plain order instead
+        e2e_pipelined, e2e_note = False, f"{type(exc).__name__}: {exc}"[:200]
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                serial_e2e_step(i)
+        stream.synchronize()
+        e2e_ms = timed(serial_e2e_step, args.steps)
+    for g in graphs + list(e2e_graphs.values()):
         g.reset()
 
     # -------- roofline of the dominant kernel --------
@@ -397,6 +493,8 @@ def run_ours(args):
                   "TFLOPs": round(layer_tflops, 2), "hbm_frac_of_measured": round(layer_gbs / hbm, 4)},
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "overlap": ("two buffer sets: step i+1's inputs copy in and step i-1's result copies out while "
+                            "step i computes") if e2e_pipelined else f"none (pipelined order failed: {e2e_note})",
                 "h2d_bytes_per_step": T * w.H * 2 + T * w.E * 4, "d2h_bytes_per_step": T * w.H * 4},
         "gpu_launches": launches,
         "eager_ms_per_step": round(eager_ms / args.steps, 5),
