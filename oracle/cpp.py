@@ -29,6 +29,12 @@ def lib() -> ctypes.CDLL:
         L.orc_pack.restype = c_int
         L.orc_pack.argtypes = [POINTER(c_float), c_int, c_int, POINTER(c_uint8), POINTER(c_uint8), c_int,
                                POINTER(c_float)]
+        L.orc_e8m0_value.restype = c_double
+        L.orc_e8m0_value.argtypes = [c_int]
+        L.orc_pack_mxfp4.restype = c_int
+        L.orc_pack_mxfp4.argtypes = [POINTER(c_float), c_int, c_int, POINTER(c_uint8), POINTER(c_uint8), c_int]
+        L.orc_decode_mxfp4.restype = c_int
+        L.orc_decode_mxfp4.argtypes = [POINTER(c_uint8), POINTER(c_uint8), c_int, c_int, c_int, POINTER(c_double)]
         L.orc_route.restype = c_int
         L.orc_route.argtypes = [POINTER(c_float), c_int, c_int, c_int, POINTER(c_int32), POINTER(c_double)]
         L.orc_permute.restype = c_int
@@ -65,6 +71,35 @@ def pack(w: np.ndarray, ld_scale: Optional[int] = None):
     if lib().orc_pack(_p(w, c_float), N, K, _p(codes, c_uint8), _p(scales, c_uint8), ld, _p(g, c_float)) != 0:
         raise ValueError("orc_pack: K must be a multiple of 16 and ld_scale >= K/16")
     return codes, scales, np.float32(g[0])
+
+
+def e8m0_value(byte: int) -> float:
+    return float(lib().orc_e8m0_value(byte))
+
+
+def pack_mxfp4(w: np.ndarray, ld_scale: Optional[int] = None):
+    """fp32 [N, K] -> (codes uint8 [N, K/2], E8M0 scales uint8 [N, ld])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    ld = K // 32 if ld_scale is None else ld_scale
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    scales = np.zeros((N, ld), dtype=np.uint8)
+    rc = lib().orc_pack_mxfp4(_p(w, c_float), N, K, _p(codes, c_uint8), _p(scales, c_uint8), ld)
+    if rc != 0:
+        raise ValueError({-1: "K must be a multiple of 32 and ld_scale >= K/32",
+                          -2: "non-finite input"}.get(rc, str(rc)))
+    return codes, scales
+
+
+def decode_mxfp4(codes: np.ndarray, scales: np.ndarray, K: int) -> np.ndarray:
+    """MXFP4 [N, K] -> fp64 values."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    N, ld = scales.shape
+    out = np.zeros((N, K), dtype=np.float64)
+    if lib().orc_decode_mxfp4(_p(codes, c_uint8), _p(scales, c_uint8), N, K, ld, _p(out, c_double)) != 0:
+        raise ValueError("orc_decode_mxfp4: bad sizes or a NaN scale byte")
+    return out
 
 
 def route(logits: np.ndarray, k: int):

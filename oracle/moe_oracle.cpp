@@ -19,6 +19,11 @@
 //   expert   G = Wg x, U = Wu x, h = G * U / (1 + exp(-G)), o = Wd h  (fp64)
 //   combine  y[t] = sum_j w_j * o_{t,j}  (fp64)
 //   pack     fp32 weights -> NVFP4 with IEEE fp32 round-to-nearest steps
+//   mxfp4    the MXFP4 expert format the pages list beside NVFP4 ("FlashML-org /
+//            FreeToken" about page, quantization formats; model guide, CPU
+//            executor formats): E2M1 elements sharing one E8M0 scale per 32,
+//            as the OCP Microscaling Formats (MX) v1.0 specification defines
+//            the format and its conversion from fp32
 //
 // Build: g++ -O2 -std=c++17 -ffp-contract=off -fopenmp -shared -fPIC
 // (oracle/build.py); -ffp-contract=off keeps every fp32 step of pack a
@@ -48,6 +53,11 @@ double e4m3_value(int byte) {
   if (e == 15 && m == 7) return std::nan("");
   const double mag = e == 0 ? std::ldexp(m / 8.0, -6) : std::ldexp(1.0 + m / 8.0, e - 7);
   return s ? -mag : mag;
+}
+
+// E8M0 (MX shared scale): 2^(byte - 127); 255 is NaN; no sign, no zero.
+double e8m0_value(int byte) {
+  return byte == 255 ? std::nan("") : std::ldexp(1.0, byte - 127);
 }
 
 struct Tables {
@@ -163,6 +173,66 @@ int orc_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int 
       }
     }
   }
+  return 0;
+}
+
+// Value of an E8M0 byte (NaN for 255).
+double orc_e8m0_value(int byte) { return e8m0_value(byte & 255); }
+
+// fp32 [N, K] -> MXFP4: codes [N, K/2] (even k in the low nibble), E8M0
+// scales [N, ld] (padding zero), one scale per 32-element block.  Per block
+// (the MX conversion of a vector):
+//   x_b = floor(log2(amax_b)) - 2     (2: the largest exponent of E2M1, whose
+//                                      largest value is 1.5 * 2^2 = 6),
+//         clamped to [-127, 127]; x_b = -127 when amax_b = 0
+//   scale byte = x_b + 127
+//   q   = E2M1(w / 2^x_b) nearest-even, saturating at 6; sign follows w.
+// Returns 0; -1 if K is not a multiple of 32 or ld < K/32; -2 on a
+// non-finite input.
+int orc_pack_mxfp4(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld) {
+  if (K % 32 || ld < K / 32) return -1;
+  for (size_t i = 0; i < size_t(N) * K; ++i)
+    if (!std::isfinite(w[i])) return -2;
+  double e2m1_pos[8];
+  for (int i = 0; i < 8; ++i) e2m1_pos[i] = tables().e2m1[i];
+  for (int n = 0; n < N; ++n) {
+    std::memset(scales + size_t(n) * ld, 0, ld);
+    for (int b = 0; b < K / 32; ++b) {
+      const float* blk = w + size_t(n) * K + 32 * b;
+      double amax = 0.0;
+      for (int i = 0; i < 32; ++i) amax = std::max(amax, double(std::fabs(blk[i])));
+      int x = -127;
+      if (amax > 0.0) {
+        int e;
+        std::frexp(amax, &e);        // amax = f * 2^e, f in [0.5, 1): floor(log2 amax) = e - 1
+        x = std::min(127, std::max(-127, (e - 1) - 2));
+      }
+      scales[size_t(n) * ld + b] = uint8_t(x + 127);
+      for (int i = 0; i < 32; i += 2) {
+        int c[2];
+        for (int h = 0; h < 2; ++h) {
+          const double v = std::ldexp(double(blk[i + h]), -x);   // exact: a power-of-two scaling in fp64
+          c[h] = round_to_grid(std::fabs(v), e2m1_pos, 8) | (std::signbit(v) ? 8 : 0);
+        }
+        codes[size_t(n) * (K / 2) + (32 * b + i) / 2] = uint8_t(c[0] | (c[1] << 4));
+      }
+    }
+  }
+  return 0;
+}
+
+// MXFP4 [N, K] -> fp64 values (exact): e2m1(code) * 2^(scale - 127).
+// Returns 0, or -1 for bad sizes or a NaN scale byte.
+int orc_decode_mxfp4(const uint8_t* codes, const uint8_t* scales, int N, int K, int ld, double* out) {
+  if (K % 32 || ld < K / 32) return -1;
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      const uint8_t sb = scales[size_t(n) * ld + k / 32];
+      if (sb == 255) return -1;
+      const uint8_t byte = codes[size_t(n) * (K / 2) + k / 2];
+      const int code = (k & 1) ? (byte >> 4) : (byte & 15);
+      out[size_t(n) * K + k] = tables().e2m1[code] * e8m0_value(sb);
+    }
   return 0;
 }
 
