@@ -10,8 +10,9 @@ import it.
 Two implementations of the same steps and readings, written apart:
   moe_oracle.cpp - plain C++ (fp64; fp32 where the format fixes it), the
                    oracle the GPU parity tests, the smoke check and the bench's
-                   CPU legs use; cpp.py is its ctypes front end, build.py
-                   compiles it with g++
+                   CPU legs use; also MXFP4 pack and decode (OCP MX v1.0) for
+                   the MXFP4 expert variant; cpp.py is its ctypes front end,
+                   build.py compiles it with g++
   nvfp4          - numpy: E2M1/E4M3 decode from bits, NVFP4 decode and pack
   moe_layer      - numpy: route, permute, SwiGLU expert FFN, combine, tolerance
 
