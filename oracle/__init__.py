@@ -15,6 +15,8 @@ Two implementations of the same steps and readings, written apart:
                    build.py compiles it with g++
   nvfp4          - numpy: E2M1/E4M3 decode from bits, NVFP4 decode and pack
   moe_layer      - numpy: route, permute, SwiGLU expert FFN, combine, tolerance
+  mxfp4          - numpy: MXFP4 (OCP MX) pack and decode, written apart from
+                   the C++ one
 
 Every function is pinned by a ``-m "not gpu"`` test against something other
 than itself (hand-worked tables, closed forms, brute force, a library routine

@@ -33,7 +33,7 @@ def test_hand_worked_blocks():
     w = np.zeros((1, 128), np.float32)
     # block 0: amax 7, floor(log2 7) = 2, shared exponent 2 - 2 = 0, scale 2^0 (byte 127)
     #   6 -> 6 (code 7); 3 -> code 5; -1.5 -> 8 | 3 = 11; 0.25: tie of 0 and 0.5 -> even index 0;
-    #   0.75: tie of 1 and 1.5?  no: of 0.5 (index 1) and 1.0 (index 2) -> even index 2 (code 2);
+    #   0.75: tie of 0.5 (index 1) and 1.0 (index 2) -> even index 2 (code 2);
     #   -0.0 -> code 8; 5: tie of 4 (index 6) and 6 (index 7) -> index 6 (code 6); 7 saturates to 6 (code 7)
     w[0, :8] = [6.0, 3.0, -1.5, 0.25, 0.75, -0.0, 5.0, 7.0]
     # block 1: amax 0.8, floor(log2 0.8) = -1, shared exponent -3, scale 1/8 (byte 124)
@@ -117,3 +117,19 @@ def test_rejects_bad_inputs():
         cpp.pack_mxfp4(bad)
     with pytest.raises(ValueError):
         cpp.decode_mxfp4(np.zeros((1, 16), np.uint8), np.full((1, 1), 255, np.uint8), 32)
+
+
+def test_numpy_and_cpp_oracles_agree_bit_for_bit():
+    """Two MXFP4 implementations written apart (numpy, C++) on random,
+    scaled, tied and saturating inputs."""
+    from oracle import mxfp4
+    g = np.random.default_rng(13)
+    w = (g.standard_normal((6, 128)) * np.float32(0.04)).astype(np.float32)
+    w[1] *= np.float32(2.0 ** 40)
+    w[2] *= np.float32(2.0 ** -60)
+    w[3, :8] = [0.25, 0.75, 5.0, 7.0, -0.0, 1e-30, -6.5, 2.5]
+    w[4, 32:64] = 0.0
+    c1, s1 = cpp.pack_mxfp4(w)
+    c2, s2 = mxfp4.pack(w)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    assert np.array_equal(cpp.decode_mxfp4(c1, s1, 128), mxfp4.decode(c2, s2, 128))
