@@ -17,6 +17,8 @@
  *   combine  -> ft_moe_combine    y[t] = sum_j w[t,j] * o[row(t,j)]
  *   format   -> ft_nvfp4_pack     fp32 weights -> NVFP4 (E2M1 + E4M3/16 + fp32)
  *   cache    -> ft_slot_*         host LRU of expert slots in a device pool
+ *   EP       -> ft_ep_plan, ft_gather_rows   experts split over ranks; the rows
+ *                                 of each rank's experts exchanged all-to-all
  *
  * Conventions (all functions):
  *   - Return an int status (FT_OK or a negative FT_ERR_*).  On FT_ERR_CUDA the
@@ -234,6 +236,63 @@ FT_API int ft_device_status(int* status, int clear);
 FT_API int ft_device_status_detail(int64_t detail[8]);
 
 /* ---------------------------------------------------------------------------
+ * Expert parallelism.  The fork's production configuration splits the experts
+ * of every MoE layer over two GPUs ("sm89-moe-offload" fork README,
+ * "Production configuration": --moe-ep-size 2 beside tensor parallelism);
+ * the pages do not say how the rows travel.  The reading used here, for G
+ * ranks with E % G == 0:
+ *   - rank r owns experts [r*E/G, (r+1)*E/G) (contiguous blocks);
+ *   - every rank routes and permutes its own T_r tokens over all E experts,
+ *     so the rows it must send to rank d are one contiguous range of its
+ *     permuted rows: [offsets_r[d*E/G], offsets_r[(d+1)*E/G]);
+ *   - the ranks exchange their expert_offsets (an all-gather of G x (E+1)
+ *     int32), then all-to-all the activation rows (ft_gather_rows with
+ *     idx = perm_src, div = k lays them out), run ft_moe_ffn_nvfp4 over their
+ *     own experts on what arrived, all-to-all the output rows back, and
+ *     combine as on one GPU.
+ * Rows arrive grouped by source rank; the plan gives the receiver a
+ * perm_src that visits them expert by expert, so the FFN reads them in
+ * place (x = the received rows, T = n_recv, k = 1, E = E/G), and the inverse
+ * map to put the outputs back in arrival order (ft_gather_rows, div = 1).
+ * Each rank's out_perm then holds, row for row, what one GPU would compute.
+ * ------------------------------------------------------------------------- */
+
+/*
+ * The exchange plan of `rank`, on the host (no CUDA calls).
+ *   all_offsets     host int32 [G][E+1]: every rank's expert_offsets from
+ *                   ft_moe_permute (row s from rank s); each row starts at 0
+ *                   and never decreases
+ *   send_rows       host int32 [G] (out): rows this rank sends to rank d
+ *   recv_rows       host int32 [G] (out): rows it receives from rank s
+ *   local_offsets   host int32 [E/G + 1] (out): group offsets of its experts
+ *                   over the received rows, expert by expert
+ *   perm_src_local  host int32 [cap] (out): row r of that grouping -> index of
+ *                   the received row (arrival order: by source rank, then as
+ *                   the source's permuted order); within an expert, rows go
+ *                   by source rank, then by the source's pair order
+ *   ret_idx         host int32 [cap] (out): the inverse of perm_src_local
+ *   *n_recv         (out) rows received = local_offsets[E/G]
+ * perm_src_local and ret_idx may both be NULL (sizes only).  Returns
+ * FT_ERR_INVALID_ARG for G < 1, E % G != 0, rank outside [0, G), malformed
+ * offsets, or n_recv > cap (after writing *n_recv and the row counts).
+ */
+FT_API int ft_ep_plan(const int32_t* all_offsets, int G, int E, int rank, int32_t* send_rows,
+                      int32_t* recv_rows, int32_t* local_offsets, int32_t* perm_src_local,
+                      int32_t* ret_idx, int cap, int32_t* n_recv);
+
+/*
+ * Row gather on the device: dst[i, :] = src[idx[i] / div, :] for i in [0, n).
+ *   src        device, n_src rows of row_bytes bytes
+ *   idx        device int32 [n]
+ *   dst        device, n rows of row_bytes bytes (out)
+ * row_bytes must be a positive multiple of 16 and src and dst 16-byte
+ * aligned; div >= 1.  An index whose row falls outside [0, n_src) sets
+ * FT_DEV_BAD_INDEX and gives a zero row.  n = 0 is a no-op.
+ */
+FT_API int ft_gather_rows(const void* src, int n_src, int row_bytes, const int32_t* idx, int div, int n,
+                          void* dst, ft_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Expert slot manager: a host-side LRU over (layer, expert) keys, mirroring
  * the pages' global LRU expert cache (FreeToken model guide, offload strategy,
  * OffloadMoeCache with per-(layer, expert) recency and a minimum-size guard;
@@ -300,7 +359,8 @@ enum {
   FT_KERNEL_PACK = 6,
   FT_KERNEL_PREP = 7,         /* work lists + activations to f16 (inside ft_moe_ffn_nvfp4) */
   FT_KERNEL_FFN_DECODE = 8,   /* decode variant: gate/up + SwiGLU + down in one launch */
-  FT_KERNEL_KINDS = 9,
+  FT_KERNEL_GATHER = 9,       /* row gather of the expert-parallel exchange */
+  FT_KERNEL_KINDS = 10,
 };
 
 typedef struct {

@@ -53,11 +53,12 @@ class SlotLayout(ctypes.Structure):
 
 
 FT_KERNEL_NAMES = ("route", "permute", "schedule", "gemm_gate_up", "gemm_down", "combine", "pack", "prep_x",
-                   "ffn_decode")
+                   "ffn_decode", "gather")
 
 
 class Profile(ctypes.Structure):
-    _fields_ = [("launches", c_int64 * 9), ("timed", c_int64 * 9), ("total_ms", ctypes.c_double * 9)]
+    _fields_ = [("launches", c_int64 * len(FT_KERNEL_NAMES)), ("timed", c_int64 * len(FT_KERNEL_NAMES)),
+                ("total_ms", ctypes.c_double * len(FT_KERNEL_NAMES))]
 
 
 class SlotStats(ctypes.Structure):
@@ -78,6 +79,9 @@ _SIGS = {
     "ft_nvfp4_pack": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "ft_device_status": (c_int, [POINTER(c_int), c_int]),
     "ft_device_status_detail": (c_int, [POINTER(c_int64)]),
+    "ft_gather_rows": (c_int, [c_void_p, c_int, c_int, c_void_p, c_int, c_int, c_void_p, c_void_p]),
+    "ft_ep_plan": (c_int, [POINTER(c_int32), c_int, c_int, c_int, POINTER(c_int32), POINTER(c_int32),
+                           POINTER(c_int32), POINTER(c_int32), POINTER(c_int32), c_int, POINTER(c_int32)]),
     "ft_slot_create": (c_int, [POINTER(c_void_p), c_int, POINTER(SlotLayout), c_void_p, c_int]),
     "ft_slot_register_host": (c_int, [c_void_p, c_int, c_int, c_void_p]),
     "ft_slot_acquire": (c_int, [c_void_p, c_int, POINTER(c_int32), c_int, c_void_p, c_int, c_void_p, c_void_p]),
@@ -149,6 +153,23 @@ def ffn_nvfp4(x, T, H, I, E, k, perm_src, offsets, slot_table, pool, layout, out
 
 def combine(out_perm, pair_to_row, w, T, k, H, y, stream) -> None:
     check(lib().ft_moe_combine(out_perm, pair_to_row, w, T, k, H, y, stream))
+
+
+def gather_rows(src, n_src, row_bytes, idx, div, n, dst, stream) -> None:
+    check(lib().ft_gather_rows(src, n_src, row_bytes, idx, div, n, dst, stream))
+
+
+def ep_plan(all_offsets, G: int, E: int, rank: int, cap: int, send_rows, recv_rows, local_offsets,
+            perm_src_local, ret_idx) -> int:
+    """ft_ep_plan on host int32 arrays (numpy or CPU torch, C-contiguous);
+    perm_src_local and ret_idx may both be None.  Returns n_recv."""
+    def p(a):
+        return None if a is None else ctypes.cast(a.ctypes.data if hasattr(a, "ctypes") else a.data_ptr(),
+                                                  POINTER(c_int32))
+    n = c_int32(0)
+    check(lib().ft_ep_plan(p(all_offsets), G, E, rank, p(send_rows), p(recv_rows), p(local_offsets),
+                           p(perm_src_local), p(ret_idx), cap, ctypes.byref(n)))
+    return int(n.value)
 
 
 def nvfp4_pack(w, N, K, codes, scales, ld_scale, global_scale, ws, stream) -> None:

@@ -137,6 +137,18 @@ extern "C" int ft_moe_combine(const void* out_perm, const int32_t* pair_to_row, 
   return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_combine");
 }
 
+extern "C" int ft_gather_rows(const void* src, int n_src, int row_bytes, const int32_t* idx, int div, int n,
+                              void* dst, ft_stream_t stream) {
+  if (n < 0 || n_src < 0 || row_bytes < 16 || row_bytes % 16 || div < 1)
+    return fail(FT_ERR_INVALID_ARG, "ft_gather_rows: need n, n_src >= 0, row_bytes a positive multiple of 16, div >= 1");
+  if (n == 0) return FT_OK;
+  if (!src || !idx || !dst) return fail(FT_ERR_INVALID_ARG, "ft_gather_rows: null pointer");
+  if ((reinterpret_cast<uintptr_t>(src) & 15) || (reinterpret_cast<uintptr_t>(dst) & 15))
+    return fail(FT_ERR_INVALID_ARG, "ft_gather_rows: src and dst must be 16-byte aligned");
+  const cudaError_t e = launch_gather_rows(src, n_src, row_bytes, idx, div, n, dst, device_sm_count(), S(stream));
+  return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_gather_rows");
+}
+
 extern "C" int ft_nvfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
                              float* global_scale, void* ws, ft_stream_t stream) {
   if (N < 1 || K < 16 || K % 16 || ld_scale < K / 16)

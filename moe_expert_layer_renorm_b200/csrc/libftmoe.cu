@@ -10,6 +10,7 @@
 #include "route.cu"
 #include "permute.cu"
 #include "combine.cu"
+#include "gather.cu"
 #include "pack.cu"
 #include "ffn.cu"
 #include "decode.cu"
@@ -17,3 +18,4 @@
 #include "api.cu"
 #include "permute_noalloc.cu"
 #include "slots.cpp"
+#include "ep.cpp"
