@@ -235,6 +235,18 @@ FT_API int ft_device_status(int* status, int clear);
  */
 FT_API int ft_device_status_detail(int64_t detail[8]);
 
+/*
+ * Test hook for the failure path: launches one CTA of two warps that wait on
+ * mbarriers nothing completes, through the bounded wait of the expert
+ * GEMMs.  Warp 0's wait gives up after ~1 s and records FT_DEV_WAIT_TIMEOUT
+ * (detail: block 0, warp 0, barrier kind 4, counter 7, unit 3) and raises
+ * the CTA's abort flag; warp 1, which starts 0.5 s later, sees the flag and
+ * leaves before its own limit.  out[w] (device int32 [2]) = 1 when warp w's
+ * wait gave up.  The kernel ends normally (no trap, no fault), so the
+ * context stays usable.  Takes one to two seconds of device time.
+ */
+FT_API int ft_selftest_wait_timeout(int32_t* out, ft_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Expert parallelism.  The fork's production configuration splits the experts
  * of every MoE layer over two GPUs ("sm89-moe-offload" fork README,

@@ -79,6 +79,7 @@ _SIGS = {
     "ft_nvfp4_pack": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "ft_device_status": (c_int, [POINTER(c_int), c_int]),
     "ft_device_status_detail": (c_int, [POINTER(c_int64)]),
+    "ft_selftest_wait_timeout": (c_int, [c_void_p, c_void_p]),
     "ft_gather_rows": (c_int, [c_void_p, c_int, c_int, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "ft_ep_plan": (c_int, [POINTER(c_int32), c_int, c_int, c_int, POINTER(c_int32), POINTER(c_int32),
                            POINTER(c_int32), POINTER(c_int32), POINTER(c_int32), c_int, POINTER(c_int32)]),
@@ -180,6 +181,11 @@ def device_status(clear: bool = True) -> int:
     v = c_int(0)
     check(lib().ft_device_status(ctypes.byref(v), 1 if clear else 0))
     return v.value
+
+
+def selftest_wait_timeout(out, stream) -> None:
+    """ft_selftest_wait_timeout: a kernel whose bounded waits run out (~1 s)."""
+    check(lib().ft_selftest_wait_timeout(out, stream))
 
 
 def device_status_detail() -> list:

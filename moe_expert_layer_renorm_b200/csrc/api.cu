@@ -178,6 +178,12 @@ extern "C" int ft_device_status(int* status, int clear) {
   return FT_OK;
 }
 
+extern "C" int ft_selftest_wait_timeout(int32_t* out, ft_stream_t stream) {
+  if (!out) return fail(FT_ERR_INVALID_ARG, "ft_selftest_wait_timeout: null pointer");
+  const cudaError_t e = launch_wait_selftest(out, S(stream));
+  return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_selftest_wait_timeout");
+}
+
 extern "C" int ft_device_status_detail(int64_t* detail) {
   if (!detail) return fail(FT_ERR_INVALID_ARG, "ft_device_status_detail: null pointer");
   cudaError_t e = cudaDeviceSynchronize();

@@ -14,6 +14,7 @@
 #include "pack.cu"
 #include "ffn.cu"
 #include "decode.cu"
+#include "selftest.cu"
 #include "ffn_host.cu"
 #include "api.cu"
 #include "permute_noalloc.cu"
