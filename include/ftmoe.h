@@ -137,6 +137,19 @@ FT_API int ft_moe_permute(const int32_t* topk_ids, int T, int k, int E,
 FT_API size_t ft_moe_permute_workspace_size(int T, int k, int E);
 
 /*
+ * ft_moe_route followed by ft_moe_permute, as one call: the outputs of both,
+ * bit for bit.  Small batches (T <= 128, T*k <= 1024, E <= 512: the decode
+ * sizes) run both steps in one kernel launch that keeps the selected ids in
+ * shared memory; other sizes launch the two calls' kernels.  Arguments are
+ * those of the two calls; ws and ws_bytes as for ft_moe_permute (no
+ * workspace is needed when T*k <= 1024).
+ */
+FT_API int ft_moe_route_permute(const float* logits, int T, int E, int k, int mode,
+                                int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                                int32_t* perm_src, int32_t* pair_to_row, void* ws, size_t ws_bytes,
+                                ft_stream_t stream);
+
+/*
  * ft_moe_permute without a workspace argument and without allocating.  The
  * pages have no counterpart of this call: it is an interface convenience.
  * Output is identical, bit for bit, to ft_moe_permute's.
@@ -372,7 +385,8 @@ enum {
   FT_KERNEL_PREP = 7,         /* work lists + activations to f16 (inside ft_moe_ffn_nvfp4) */
   FT_KERNEL_FFN_DECODE = 8,   /* decode variant: gate/up + SwiGLU + down in one launch */
   FT_KERNEL_GATHER = 9,       /* row gather of the expert-parallel exchange */
-  FT_KERNEL_KINDS = 10,
+  FT_KERNEL_ROUTE_PERMUTE = 10, /* route and permute in one launch (small batches) */
+  FT_KERNEL_KINDS = 11,
 };
 
 typedef struct {

@@ -53,7 +53,7 @@ class SlotLayout(ctypes.Structure):
 
 
 FT_KERNEL_NAMES = ("route", "permute", "schedule", "gemm_gate_up", "gemm_down", "combine", "pack", "prep_x",
-                   "ffn_decode", "gather")
+                   "ffn_decode", "gather", "route_permute")
 
 
 class Profile(ctypes.Structure):
@@ -71,6 +71,8 @@ _SIGS = {
     "ft_moe_permute": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                c_void_p]),
     "ft_moe_permute_workspace_size": (c_size_t, [c_int, c_int, c_int]),
+    "ft_moe_route_permute": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_size_t, c_void_p]),
     "ft_moe_permute_noalloc": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "ft_moe_ffn_nvfp4": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
                                  c_void_p, POINTER(SlotLayout), c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -134,6 +136,11 @@ def permute_workspace_size(T, k, E) -> int:
 
 def permute(ids, T, k, E, offsets, perm_src, pair_to_row, ws, ws_bytes, stream) -> None:
     check(lib().ft_moe_permute(ids, T, k, E, offsets, perm_src, pair_to_row, ws, ws_bytes, stream))
+
+
+def route_permute(logits, T, E, k, mode, ids, w, offsets, perm_src, pair_to_row, ws, ws_bytes, stream) -> None:
+    check(lib().ft_moe_route_permute(logits, T, E, k, mode, ids, w, offsets, perm_src, pair_to_row, ws, ws_bytes,
+                                     stream))
 
 
 def permute_noalloc(ids, T, k, E, offsets, perm_src, pair_to_row, stream) -> None:

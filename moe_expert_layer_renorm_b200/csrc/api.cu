@@ -92,6 +92,28 @@ extern "C" int ft_moe_permute(const int32_t* ids, int T, int k, int E, int32_t* 
   return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_permute");
 }
 
+extern "C" int ft_moe_route_permute(const float* logits, int T, int E, int k, int mode, int32_t* ids, float* w,
+                                    int32_t* offsets, int32_t* perm_src, int32_t* pair_to_row, void* ws,
+                                    size_t ws_bytes, ft_stream_t stream) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32 || (mode != 0 && mode != 1) ||
+      (long long)T * k > (1LL << 30))
+    return fail(FT_ERR_INVALID_ARG, "ft_moe_route_permute: need 1 <= k <= min(E, 32), E <= 1024, mode 0 or 1");
+  if (!offsets) return fail(FT_ERR_INVALID_ARG, "ft_moe_route_permute: null pointer");
+  if (T == 0) {
+    const cudaError_t e = cudaMemsetAsync(offsets, 0, size_t(E + 1) * sizeof(int32_t), S(stream));
+    return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_route_permute");
+  }
+  if (!logits || !ids || !w || !perm_src || !pair_to_row)
+    return fail(FT_ERR_INVALID_ARG, "ft_moe_route_permute: null pointer");
+  if (!route_permute_fused_fits(T, k, E)) {
+    const int r = ft_moe_route(logits, T, E, k, mode, ids, w, stream);
+    return r != FT_OK ? r : ft_moe_permute(ids, T, k, E, offsets, perm_src, pair_to_row, ws, ws_bytes, stream);
+  }
+  const cudaError_t e =
+      launch_route_permute_small(logits, T, E, k, mode, ids, w, offsets, perm_src, pair_to_row, S(stream));
+  return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_route_permute");
+}
+
 static bool ffn_shape_ok(int H, int I, int E, int k) {
   return H >= 256 && I >= 256 && H % 64 == 0 && I % 64 == 0 && E >= 1 && E <= 1024 && k >= 1 && k <= E &&
          H <= 65536 && I <= 65536;

@@ -147,6 +147,89 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __r
   }
 }
 
+// Route and permute in one CTA for small batches (T <= kFusedMaxT tokens,
+// T*k <= kPermChunk pairs, E <= kFusedMaxE): each warp routes tokens with the
+// same per-token code as route_kernel (so the same ids and weight bits), the
+// selected ids stay in shared memory, and the counting sort of
+// permute_small_kernel reads them from there.  Saves a launch and the ids'
+// round trip through global memory on the decode path.
+constexpr int kFusedMaxT = 128;
+constexpr int kFusedMaxE = 512;
+
+// One warp places pairs 0 .. P-1 in order; ids in shared memory, cursor[e] the
+// next row of expert e.
+__device__ void scatter_smem_warp(const int* s_ids, int P, int* cursor, int32_t* __restrict__ perm_src,
+                                  int32_t* __restrict__ pair_to_row) {
+  const int lane = threadIdx.x & 31;
+  for (int base = 0; base < P; base += 32) {
+    const int p = base + lane;
+    const int e = p < P ? s_ids[p] : -1;
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int leader = __ffs(peers) - 1;
+    const int row = e >= 0 ? cursor[e] + rank : -1;
+    __syncwarp();
+    if (e >= 0 && lane == leader) cursor[e] += __popc(peers);
+    __syncwarp();
+    if (row >= 0 && row < P) {
+      perm_src[row] = p;
+      pair_to_row[p] = row;
+    }
+  }
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(1024) route_permute_small_kernel(const float* __restrict__ logits, int T, int E,
+                                                                   int k, int mode, int32_t* __restrict__ ids,
+                                                                   float* __restrict__ wts,
+                                                                   int32_t* __restrict__ offsets,
+                                                                   int32_t* __restrict__ perm_src,
+                                                                   int32_t* __restrict__ pair_to_row) {
+  pdl_enter();
+  __shared__ int s_ids[kPermChunk];
+  __shared__ int cnt[kFusedMaxE];
+  __shared__ int warp_sums[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  for (int t = warp; t < T; t += nwarps) {
+    int sel_id;
+    float w;
+    route_token<NPL>(logits + size_t(t) * E, E, k, mode, lane, sel_id, w);
+    if (lane < k) {
+      ids[size_t(t) * k + lane] = sel_id;
+      wts[size_t(t) * k + lane] = w;
+      s_ids[t * k + lane] = sel_id;
+    }
+  }
+  __syncthreads();
+  const int P = T * k;
+  for (int p = threadIdx.x; p < P; p += blockDim.x) atomicAdd(&cnt[s_ids[p]], 1);
+  __syncthreads();
+  const int e = threadIdx.x;   // E <= kFusedMaxE <= blockDim.x: one expert per thread
+  const int c = e < E ? cnt[e] : 0;
+  const int ex = block_exclusive_scan(c, warp_sums);
+  if (e < E) { offsets[e] = ex; cnt[e] = ex; }
+  if (e == E - 1) offsets[E] = ex + c;
+  __syncthreads();
+  if (warp == 0) scatter_smem_warp(s_ids, P, cnt, perm_src, pair_to_row);
+}
+
+static bool route_permute_fused_fits(int T, int k, int E) {
+  return T >= 1 && T <= kFusedMaxT && T * k <= kPermChunk && E <= kFusedMaxE;
+}
+
+static cudaError_t launch_route_permute_small(const float* logits, int T, int E, int k, int mode, int32_t* ids,
+                                              float* w, int32_t* offsets, int32_t* perm_src, int32_t* pair_to_row,
+                                              cudaStream_t s) {
+  const int npl = (E + 31) / 32;
+  ProfileScope prof(FT_KERNEL_ROUTE_PERMUTE, s);
+  auto kern = npl <= 1 ? route_permute_small_kernel<1> : npl <= 2 ? route_permute_small_kernel<2>
+             : npl <= 4 ? route_permute_small_kernel<4> : npl <= 8 ? route_permute_small_kernel<8>
+             : route_permute_small_kernel<16>;
+  return launch_pdl(kern, dim3(1), dim3(1024), 0, s, logits, T, E, k, mode, ids, w, offsets, perm_src,
+                    pair_to_row);
+}
+
 static size_t permute_ws_bytes(int T, int k, int E) {
   const long long P = (long long)T * k;
   const long long nchunks = (P + kPermChunk - 1) / kPermChunk;

@@ -12,15 +12,12 @@
 
 namespace ftmoe {
 
+// The top-k and weights of one token, computed by one warp: lane j < k gets
+// the j-th selected expert and its weight.  `row` points at the token's E
+// logits.
 template <int NPL>  // logits per lane = ceil(E / 32)
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                     int mode, int32_t* __restrict__ ids,
-                                                     float* __restrict__ wts) {
-  pdl_enter();
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  if (t >= T) return;
-  const float* row = logits + size_t(t) * E;
+__device__ __forceinline__ void route_token(const float* __restrict__ row, int E, int k, int mode, int lane,
+                                            int& sel_id_out, float& w_out) {
   float v[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
@@ -79,7 +76,22 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
     w = p / s;
   }
-  if (mine) {
+  sel_id_out = sel_id;
+  w_out = w;
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                     int mode, int32_t* __restrict__ ids,
+                                                     float* __restrict__ wts) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (t >= T) return;
+  int sel_id;
+  float w;
+  route_token<NPL>(logits + size_t(t) * E, E, k, mode, lane, sel_id, w);
+  if (lane < k) {
     ids[size_t(t) * k + lane] = sel_id;
     wts[size_t(t) * k + lane] = w;
   }

@@ -68,8 +68,9 @@ class MoELayer:
     """Buffers and calls for one MoE FFN layer of fixed (T, E, k, H, I)."""
 
     def __init__(self, T: int, E: int, k: int, H: int, I: int, mode: int = _lib.FT_ROUTE_SOFTMAX_RENORM,
-                 device="cuda"):
+                 device="cuda", fused_front: bool = False):
         self.T, self.E, self.k, self.H, self.I, self.mode = T, E, k, H, I, mode
+        self.fused_front = fused_front   # route + permute through ft_moe_route_permute
         P = T * k
         dev = torch.device(device)
         i32 = dict(dtype=torch.int32, device=dev)
@@ -93,6 +94,11 @@ class MoELayer:
         _lib.permute(self.ids.data_ptr(), self.T, self.k, self.E, self.offsets.data_ptr(), self.perm_src.data_ptr(),
                      self.pair_to_row.data_ptr(), self.perm_ws.data_ptr(), self.perm_ws_bytes, _stream(stream))
 
+    def route_permute(self, logits: torch.Tensor, stream=None) -> None:
+        _lib.route_permute(logits.data_ptr(), self.T, self.E, self.k, self.mode, self.ids.data_ptr(),
+                           self.w.data_ptr(), self.offsets.data_ptr(), self.perm_src.data_ptr(),
+                           self.pair_to_row.data_ptr(), self.perm_ws.data_ptr(), self.perm_ws_bytes, _stream(stream))
+
     def ffn(self, x: torch.Tensor, slot_table: torch.Tensor, pool: ExpertPool, stream=None) -> None:
         _lib.ffn_nvfp4(x.data_ptr(), self.T, self.H, self.I, self.E, self.k, self.perm_src.data_ptr(),
                        self.offsets.data_ptr(), slot_table.data_ptr(), pool.ptr, pool.layout,
@@ -108,8 +114,11 @@ class MoELayer:
         assert x.dtype == torch.bfloat16 and x.shape == (self.T, self.H) and x.is_contiguous()
         assert logits.dtype == torch.float32 and logits.shape == (self.T, self.E) and logits.is_contiguous()
         assert slot_table.dtype == torch.int32 and slot_table.numel() == self.E
-        self.route(logits, stream)
-        self.permute(stream)
+        if self.fused_front:
+            self.route_permute(logits, stream)
+        else:
+            self.route(logits, stream)
+            self.permute(stream)
         self.ffn(x, slot_table, pool, stream)
         self.combine(stream)
         return self.y

@@ -54,7 +54,7 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
 
 
 def run_gpu(w: inputs.Workload, T: Optional[int] = None, layer: int = 0, pool=None, slot_table=None,
-            li: Optional[inputs.LayerInputs] = None, expect_status: int = 0) -> GpuRun:
+            li: Optional[inputs.LayerInputs] = None, expect_status: int = 0, fused_front: bool = False) -> GpuRun:
     li = li or inputs.make_layer_inputs(w, layer, T)
     T = li.x_bits.shape[0]
     if pool is None:
@@ -62,7 +62,7 @@ def run_gpu(w: inputs.Workload, T: Optional[int] = None, layer: int = 0, pool=No
     x = torch.from_numpy(li.x_bits.view(np.int16)).view(torch.bfloat16).cuda()
     logits = torch.from_numpy(li.logits).cuda()
     st = torch.from_numpy(np.asarray(slot_table, dtype=np.int32)).cuda()
-    lay = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode)
+    lay = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, fused_front=fused_front)
     # NaN in every intermediate the library writes before reading: an element
     # read before it is written (a missed dependency) shows up in y
     lay.ffn_ws.fill_(0xFF)
