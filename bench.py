@@ -48,6 +48,7 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"], help="expert weight format")
     ap.add_argument("--slot-churn", nargs="?", const="decode", default=None, choices=["decode", "prefill_stream"],
                     help="measure the expert-cache miss path (pinned host banks, LRU slot manager) instead: "
                          "domain-rotation decode steps, or prefill layers streamed through a two-layer pool")
@@ -68,12 +69,17 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def bytes_per_expert(H: int, I: int) -> int:
-    """Algorithmic NVFP4 bytes of one expert: codes + unpadded scales + 3 fp32 globals."""
+def bytes_per_expert(H: int, I: int, fmt: str = "nvfp4") -> int:
+    """Algorithmic bytes of one expert: codes + unpadded scales (+ 3 fp32
+    globals for NVFP4; MXFP4 has one E8M0 byte per 32 values and no global)."""
+    if fmt == "mxfp4":
+        return 3 * (H * I // 2 + H * I // 32)
     return 3 * (H * I // 2 + H * I // 16) + 12
 
 
-def gate_up_bytes_per_expert(H: int, I: int) -> int:
+def gate_up_bytes_per_expert(H: int, I: int, fmt: str = "nvfp4") -> int:
+    if fmt == "mxfp4":
+        return 2 * (H * I // 2 + H * I // 32)
     return 2 * (H * I // 2 + H * I // 16) + 8
 
 
@@ -274,7 +280,8 @@ def run_ours(args):
     # slots are permuted), as the layers of a model share an expert cache
     S = max(w.slots, R * w.E)
     order = np.random.default_rng([w.seed, rank, 9]).permutation(S) if w.permuted_slots else np.arange(S)
-    pool = ExpertPool(w.H, w.I, S, device=dev)
+    pool = ExpertPool(w.H, w.I, S, device=dev,
+                      fmt=_lib.FT_SCALE_MXFP4 if args.fmt == "mxfp4" else _lib.FT_SCALE_NVFP4)
     layers = []
     for l in range(R):
         s = rank_layer_seed(w, rank, l)
@@ -439,14 +446,14 @@ def run_ours(args):
     mean_distinct = sum(d * n for d, n in zip(distinct, steps_per_layer)) / args.steps
     P = T * w.k
     flops_step = 6.0 * w.H * w.I * P
-    decode_like = flops_step / (mean_distinct * bytes_per_expert(w.H, w.I)) < 200
+    decode_like = flops_step / (mean_distinct * bytes_per_expert(w.H, w.I, args.fmt)) < 200
     if dom_name == "ffn_decode":
         # both GEMMs in one launch: the three weight tensors of every expert hit,
         # the token rows in (bf16) and the expert outputs out (fp32)
-        alg_bytes = mean_distinct * bytes_per_expert(w.H, w.I) + T * w.H * 2 + P * w.H * 4
+        alg_bytes = mean_distinct * bytes_per_expert(w.H, w.I, args.fmt) + T * w.H * 2 + P * w.H * 4
         alg_flops = 6.0 * w.H * w.I * P
     elif dom_name == "gemm_gate_up":
-        alg_bytes = mean_distinct * gate_up_bytes_per_expert(w.H, w.I) + T * w.H * 2 + P * w.I * 2
+        alg_bytes = mean_distinct * gate_up_bytes_per_expert(w.H, w.I, args.fmt) + T * w.H * 2 + P * w.I * 2
         alg_flops = 4.0 * w.H * w.I * P
     else:
         alg_bytes = mean_distinct * (w.H * w.I // 2 + w.H * w.I // 16 + 4) + P * w.I * 2 + P * w.H * 4
@@ -472,12 +479,12 @@ def run_ours(args):
     ms_per_step = elapsed_ms / args.steps
     value = world * T * args.steps / (elapsed_ms * 1e-3)
     e2e_value = world * T * args.steps / (e2e_ms * 1e-3)
-    layer_gbs = mean_distinct * bytes_per_expert(w.H, w.I) / (ms_per_step * 1e-3) / 1e9
+    layer_gbs = mean_distinct * bytes_per_expert(w.H, w.I, args.fmt) / (ms_per_step * 1e-3) / 1e9
     layer_tflops = flops_step / (ms_per_step * 1e-3) / 1e12
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(layers[0], w, T, args.cpu_sample_tokens)
+        cpu = cpu_baseline(layers[0], w, T, args.cpu_sample_tokens, args.fmt)
 
     if world > 1:
         dist.destroy_process_group()
@@ -486,9 +493,9 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 weights, f16 MMA operands, fp32 accumulate",
+        "scaling": "weak", "vs_baseline": None, "dtype": f"{args.fmt} weights, f16 MMA operands, fp32 accumulate",
         "data": "synthetic (seeded N(0,1) activations, N(0,sigma) logits, N(0,0.02) weights packed to NVFP4)",
-        "config": workload_config(w, R, S, world, mean_distinct),
+        "config": dict(workload_config(w, R, S, world, mean_distinct), format=args.fmt),
         "layer": {"distinct_experts": round(mean_distinct, 2), "weight_GBps": round(layer_gbs, 1),
                   "TFLOPs": round(layer_tflops, 2), "hbm_frac_of_measured": round(layer_gbs / hbm, 4)},
         "roofline": roof,
@@ -512,7 +519,7 @@ def oracle_threads() -> int:
     return int(v) if v.isdigit() and int(v) > 0 else (os.cpu_count() or 1)
 
 
-def cpu_baseline(L, w, T, n_tokens):
+def cpu_baseline(L, w, T, n_tokens, fmt="nvfp4"):
     """The C++ oracle (as it stands) on a bounded sample of the same layer:
     the first n tokens, repeated until about 10 s of host time."""
     from oracle import cpp
@@ -533,11 +540,12 @@ def cpu_baseline(L, w, T, n_tokens):
     while dt < 10.0 and reps < 50:
         t0 = time.perf_counter()
         cpp.moe_layer(li.x_bits, li.logits, w.k, table, buf, pool.slot_bytes, list(Lo.codes_off),
-                      list(Lo.scales_off), list(Lo.global_off), list(Lo.ld_scale), w.H, w.I, tokens=np.arange(n))
+                      list(Lo.scales_off), list(Lo.global_off), list(Lo.ld_scale), w.H, w.I, tokens=np.arange(n),
+                      fmt=int(Lo.scale_format))
         dt += time.perf_counter() - t0
         reps += 1
     return {"value": round(n * reps / dt, 3), "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{n} tokens of one {w.name} layer x {reps} (C++ oracle: route, NVFP4 decode from the "
+            "sample": f"{n} tokens of one {w.name} layer x {reps} (C++ oracle: route, {fmt.upper()} decode from the "
                       f"bytes of the {len(need)} experts they select, fp64 SwiGLU FFN, combine); {dt:.2f} s",
             "host_cpus": os.cpu_count()}
 
@@ -584,7 +592,15 @@ def run_reference(args):
         if e not in slots:
             b = np.zeros(Lo["slot_bytes"], np.uint8)
             for mat, (N, K) in enumerate(((w.I, w.H), (w.I, w.H), (w.H, w.I))):
-                c, sc, g = cpp.pack(inputs.make_weight_fp32_host(N, K, s, e, mat), Lo["ld_scale"][mat])
+                wt = inputs.make_weight_fp32_host(N, K, s, e, mat)
+                if args.fmt == "mxfp4":   # E8M0 bytes at both of their 16-K positions; no global
+                    c, sc32 = cpp.pack_mxfp4(wt)
+                    sc = np.zeros((N, Lo["ld_scale"][mat]), np.uint8)
+                    sc[:, 0:K // 16:2] = sc32
+                    sc[:, 1:K // 16:2] = sc32
+                    g = np.float32(1.0)
+                else:
+                    c, sc, g = cpp.pack(wt, Lo["ld_scale"][mat])
                 b[Lo["codes_off"][mat]:Lo["codes_off"][mat] + c.size] = c.reshape(-1)
                 b[Lo["scales_off"][mat]:Lo["scales_off"][mat] + sc.size] = sc.reshape(-1)
                 b[Lo["global_off"][mat]:Lo["global_off"][mat] + 4] = np.frombuffer(np.float32(g).tobytes(), np.uint8)
@@ -600,7 +616,7 @@ def run_reference(args):
         table[need] = np.arange(len(need), dtype=np.int32)
         t0 = time.perf_counter()
         cpp.moe_layer(li.x_bits, li.logits, w.k, table, buf, Lo["slot_bytes"], Lo["codes_off"], Lo["scales_off"],
-                      Lo["global_off"], Lo["ld_scale"], w.H, w.I, tokens=tok)
+                      Lo["global_off"], Lo["ld_scale"], w.H, w.I, tokens=tok, fmt=1 if args.fmt == "mxfp4" else 0)
         return time.perf_counter() - t0
 
     # size each step's sample so that warm-up and timed steps together take
@@ -619,8 +635,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w, R, max(w.slots, R * w.E), world,
-                                                        inputs.expected_distinct_experts(w.T, w.E, w.k)),
+        "data": "synthetic", "config": dict(format=args.fmt, **workload_config(
+            w, R, max(w.slots, R * w.E), world, inputs.expected_distinct_experts(w.T, w.E, w.k))),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": f"{n} tokens of one {w.name} layer per step"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -99,13 +99,27 @@ typedef struct {
   int64_t global_off[3];
   int64_t slot_bytes;
   int32_t num_slots;      /* slots in the pool the layout describes */
-  int32_t reserved;
+  int32_t scale_format;   /* FT_SCALE_NVFP4 or FT_SCALE_MXFP4 */
 } ft_nvfp4_slot_layout;
+
+/* How a slot's scale bytes and global scales read.
+ *   FT_SCALE_NVFP4: one E4M3 scale per 16 K of a row; the tensor's fp32
+ *                   global scale multiplies every value.
+ *   FT_SCALE_MXFP4: one E8M0 scale 2^(s - 127) per 32 K of a row (OCP MX),
+ *                   stored twice (as if per 16 K) so that both formats share
+ *                   every offset and stride; the global holds a power of two
+ *                   2^t chosen at pack time, which the kernels divide out of
+ *                   the dequantised values and multiply back in fp32 (the
+ *                   values are e2m1 * 2^(s - 127), the global only keeps the
+ *                   f16 dequantisation exact). */
+enum { FT_SCALE_NVFP4 = 0, FT_SCALE_MXFP4 = 1 };
 
 /* Fill *out with the canonical layout for hidden size H, intermediate I and
  * num_slots slots.  H and I must be multiples of 64.  Returns FT_OK or
  * FT_ERR_INVALID_ARG. */
 FT_API int ft_nvfp4_slot_layout_init(int H, int I, int num_slots, ft_nvfp4_slot_layout* out);
+/* The same layout with scale_format = FT_SCALE_MXFP4 (identical offsets). */
+FT_API int ft_mxfp4_slot_layout_init(int H, int I, int num_slots, ft_nvfp4_slot_layout* out);
 
 /*
  * Router: per token t, the k experts with the largest logits (descending;
@@ -229,6 +243,25 @@ FT_API int ft_moe_combine(const void* out_perm, const int32_t* pair_to_row, cons
  * The destinations may point inside a slot (see ft_nvfp4_slot_layout).
  */
 FT_API int ft_nvfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
+                  float* global_scale, void* ws, ft_stream_t stream);
+
+/*
+ * MXFP4 pack of one fp32 tensor [N, K] (K % 32 == 0): the OCP Microscaling
+ * (MX) conversion, which the pages name as an expert format beside NVFP4
+ * ("FlashML-org / FreeToken" about page, quantization formats) without
+ * defining it.  Per 32-block b of a row:
+ *   x_b = floor(log2 amax_b) - 2, clamped to [-127, 127]; -127 if amax_b = 0
+ *   scale byte s_b = x_b + 127, written at scales[row][2b] and [2b + 1]
+ *   q   = E2M1_rne_sat(w / 2^x_b), sign following w
+ * and for the tensor t = max_b x_b - 13 (0 if the tensor is all zero):
+ *   *global_scale = 2^t  (so that every e2m1 * 2^(x_b - t) the kernels form
+ *                         in f16 stays below 2^16; a block more than 2^36
+ *                         below the tensor's largest would lose values to f16
+ *                         underflow: the kernel then records FT_DEV_F16_RANGE)
+ * Arguments as for ft_nvfp4_pack (ld_scale >= K/16: the scales are stored at
+ * the NVFP4 granularity).  Returns FT_OK, FT_ERR_INVALID_ARG or FT_ERR_CUDA.
+ */
+FT_API int ft_mxfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
                   float* global_scale, void* ws, ft_stream_t stream);
 
 /*

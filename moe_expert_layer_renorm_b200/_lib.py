@@ -48,7 +48,7 @@ class SlotLayout(ctypes.Structure):
         ("global_off", c_int64 * 3),
         ("slot_bytes", c_int64),
         ("num_slots", c_int32),
-        ("reserved", c_int32),
+        ("scale_format", c_int32),
     ]
 
 
@@ -67,6 +67,7 @@ class SlotStats(ctypes.Structure):
 
 _SIGS = {
     "ft_nvfp4_slot_layout_init": (c_int, [c_int, c_int, c_int, POINTER(SlotLayout)]),
+    "ft_mxfp4_slot_layout_init": (c_int, [c_int, c_int, c_int, POINTER(SlotLayout)]),
     "ft_moe_route": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "ft_moe_permute": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                c_void_p]),
@@ -79,6 +80,7 @@ _SIGS = {
     "ft_moe_ffn_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "ft_moe_combine": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
     "ft_nvfp4_pack": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
+    "ft_mxfp4_pack": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "ft_device_status": (c_int, [POINTER(c_int), c_int]),
     "ft_device_status_detail": (c_int, [POINTER(c_int64)]),
     "ft_selftest_wait_timeout": (c_int, [c_void_p, c_void_p]),
@@ -120,9 +122,13 @@ def check(code: int) -> None:
         raise FtError(code, lib().ft_last_error().decode())
 
 
-def slot_layout(H: int, I: int, num_slots: int) -> SlotLayout:
+FT_SCALE_NVFP4, FT_SCALE_MXFP4 = 0, 1
+
+
+def slot_layout(H: int, I: int, num_slots: int, fmt: int = FT_SCALE_NVFP4) -> SlotLayout:
     L = SlotLayout()
-    check(lib().ft_nvfp4_slot_layout_init(H, I, num_slots, ctypes.byref(L)))
+    init = lib().ft_mxfp4_slot_layout_init if fmt == FT_SCALE_MXFP4 else lib().ft_nvfp4_slot_layout_init
+    check(init(H, I, num_slots, ctypes.byref(L)))
     return L
 
 
@@ -182,6 +188,10 @@ def ep_plan(all_offsets, G: int, E: int, rank: int, cap: int, send_rows, recv_ro
 
 def nvfp4_pack(w, N, K, codes, scales, ld_scale, global_scale, ws, stream) -> None:
     check(lib().ft_nvfp4_pack(w, N, K, codes, scales, ld_scale, global_scale, ws, stream))
+
+
+def mxfp4_pack(w, N, K, codes, scales, ld_scale, global_scale, ws, stream) -> None:
+    check(lib().ft_mxfp4_pack(w, N, K, codes, scales, ld_scale, global_scale, ws, stream))
 
 
 def device_status(clear: bool = True) -> int:

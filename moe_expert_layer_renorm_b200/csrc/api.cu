@@ -56,8 +56,15 @@ extern "C" int ft_nvfp4_slot_layout_init(int H, int I, int num_slots, ft_nvfp4_s
   }
   off = a256(off + 12);
   L.slot_bytes = off;
+  L.scale_format = FT_SCALE_NVFP4;
   *out = L;
   return FT_OK;
+}
+
+extern "C" int ft_mxfp4_slot_layout_init(int H, int I, int num_slots, ft_nvfp4_slot_layout* out) {
+  const int rc = ft_nvfp4_slot_layout_init(H, I, num_slots, out);
+  if (rc == FT_OK) out->scale_format = FT_SCALE_MXFP4;
+  return rc;
 }
 
 extern "C" int ft_moe_route(const float* logits, int T, int E, int k, int mode, int32_t* ids, float* w,
@@ -134,8 +141,10 @@ extern "C" int ft_moe_ffn_nvfp4(const void* x, int T, int H, int I, int E, int k
   if (!x || !perm_src || !expert_offsets || !slot_table || !slot_pool || !layout || !out_perm || !ws)
     return fail(FT_ERR_INVALID_ARG, "ft_moe_ffn_nvfp4: null pointer");
   if (layout->H != H || layout->I != I || layout->num_slots < 1 || layout->num_slots > (1 << 21) ||
-      layout->slot_bytes % 256)
-    return fail(FT_ERR_INVALID_ARG, "ft_moe_ffn_nvfp4: layout does not match H, I (or has more than 2^21 slots)");
+      layout->slot_bytes % 256 ||
+      (layout->scale_format != FT_SCALE_NVFP4 && layout->scale_format != FT_SCALE_MXFP4))
+    return fail(FT_ERR_INVALID_ARG,
+                "ft_moe_ffn_nvfp4: layout does not match H, I (or has more than 2^21 slots, or an unknown format)");
   if ((reinterpret_cast<uintptr_t>(slot_pool) & 255) || (reinterpret_cast<uintptr_t>(ws) & 255) ||
       (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(out_perm) & 15))
     return fail(FT_ERR_INVALID_ARG, "ft_moe_ffn_nvfp4: misaligned pointer");
@@ -180,6 +189,17 @@ extern "C" int ft_nvfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8
     return fail(FT_ERR_INVALID_ARG, "ft_nvfp4_pack: w must be 16-byte and codes 8-byte aligned");
   const cudaError_t e = launch_pack(w, N, K, codes, scales, ld_scale, global_scale, ws, S(stream));
   return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_nvfp4_pack");
+}
+
+extern "C" int ft_mxfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
+                             float* global_scale, void* ws, ft_stream_t stream) {
+  if (N < 1 || K < 16 || K % 32 || ld_scale < K / 16)
+    return fail(FT_ERR_INVALID_ARG, "ft_mxfp4_pack: need N >= 1, K a multiple of 32, ld_scale >= K/16");
+  if (!w || !codes || !scales || !global_scale || !ws) return fail(FT_ERR_INVALID_ARG, "ft_mxfp4_pack: null pointer");
+  if ((reinterpret_cast<uintptr_t>(w) & 15) || (reinterpret_cast<uintptr_t>(codes) & 7) || ((K / 2) % 8))
+    return fail(FT_ERR_INVALID_ARG, "ft_mxfp4_pack: w must be 16-byte and codes 8-byte aligned");
+  const cudaError_t e = launch_pack_mxfp4(w, N, K, codes, scales, ld_scale, global_scale, ws, S(stream));
+  return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_mxfp4_pack");
 }
 
 extern "C" int ft_device_status(int* status, int clear) {

@@ -145,8 +145,8 @@ __device__ __forceinline__ int dec_row_hi(int gemm, int w, int g) {
 }
 
 // One 256-K stage for this warp: its 16 rows x 256 K x NT token tiles of 8.
-template <int NT>
-__device__ __forceinline__ void dec_stage(const uint8_t* st, int r_lo, int r_hi, int g, int t,
+template <int NT, int FMT>
+__device__ __forceinline__ void dec_stage(const uint8_t* st, int r_lo, int r_hi, int g, int t, int blo, int bhi,
                                           float (&acc)[NT][4]) {
   const uint8_t* bst = st + kDecWStageBytes;
 #pragma unroll
@@ -160,8 +160,8 @@ __device__ __forceinline__ void dec_stage(const uint8_t* st, int r_lo, int r_hi,
     const uint32_t wlo[4] = {clo.x, clo.y, clo.z, clo.w};
     const uint32_t whi[4] = {chi.x, chi.y, chi.z, chi.w};
     // the thread's 32 K span two 16-K scale blocks: words 0, 1 and words 2, 3
-    const uint32_t sl2[2] = {e4m3_pair_to_f16x2(slo & 0xFFu), e4m3_pair_to_f16x2(slo >> 8)};
-    const uint32_t sh2[2] = {e4m3_pair_to_f16x2(shi & 0xFFu), e4m3_pair_to_f16x2(shi >> 8)};
+    const uint32_t sl2[2] = {scale_pair_to_f16x2<FMT>(slo & 0xFFu, blo), scale_pair_to_f16x2<FMT>(slo >> 8, blo)};
+    const uint32_t sh2[2] = {scale_pair_to_f16x2<FMT>(shi & 0xFFu, bhi), scale_pair_to_f16x2<FMT>(shi >> 8, bhi)};
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {   // word wd: 8 K = two MMA steps
       const int cb = (t & 1) * 4 + wd;   // the token values of those 8 K: 16-byte chunk of the box row
@@ -271,12 +271,21 @@ constexpr int kTagUnit = 10;
 // loop, so a CTA takes a new unit from the queue only when it has finished
 // computing the one before the current one: no CTA hoards small units while
 // others idle.  Returns false if a wait gave up (the kernel then winds down).
-template <int NT>
+template <int NT, int FMT>
 __device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem, uint64_t* full, uint64_t* empty,
                          const Abort& ab, uint64_t* unit_free, const int4* unit_ent, uint64_t* hpub, int* hcount,
                          int gu, uint32_t& si, int q, int w, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int r_lo = dec_row_lo(d.gemm, w, g), r_hi = dec_row_hi(d.gemm, w, g);
+  // MXFP4: the power of two each matrix's global takes out of its scales
+  // (gate/up: gate rows lo, up rows hi; down: both)
+  int blo = 0, bhi = 0;
+  if (FMT == FT_SCALE_MXFP4) {
+    const FfnParams& G = p.g[d.gemm];
+    const uint8_t* sbase = G.pool + size_t(d.slot) * size_t(G.slot_bytes);
+    blo = mx_bias(__ldg(reinterpret_cast<const float*>(sbase + G.global_off[0])));
+    bhi = mx_bias(__ldg(reinterpret_cast<const float*>(sbase + G.global_off[1])));
+  }
   // gate/up: the factors undoing the token rows' prescale, loaded now, used in the epilogue
   float ts[NT][2];
 #pragma unroll
@@ -295,7 +304,7 @@ __device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem,
   for (int ws = d.ws0; ws < d.ws1; ++ws, ++si) {
     const int s = si % kDecStages;
     if (!__all_sync(0xFFFFFFFFu, ab.wait(&full[s], (si / kDecStages) & 1, kTagWFull, si, q))) return false;
-    dec_stage<NT>(smem + s * kDecStageBytes, r_lo, r_hi, g, t, acc);
+    dec_stage<NT, FMT>(smem + s * kDecStageBytes, r_lo, r_hi, g, t, blo, bhi, acc);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
@@ -348,6 +357,7 @@ __device__ void dec_drain(uint64_t* full, uint32_t si) {
   }
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(kDecThreads, 1)
 ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c0,
                   const __grid_constant__ CUtensorMap tm_s0, const __grid_constant__ CUtensorMap tm_c1,
@@ -507,25 +517,27 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
       const DecUnit d = decode_unit(p, q, n1, udesc[us]);
       const int gu = d.gemm == 0 ? ngu++ : -1;
       const bool ok =
-          d.nr > 8 ? dec_unit<2>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], hpub, hcount, gu, si, q, warp, lane)
-                   : dec_unit<1>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], hpub, hcount, gu, si, q, warp, lane);
+          d.nr > 8 ? dec_unit<2, FMT>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], hpub, hcount, gu, si, q, warp, lane)
+                   : dec_unit<1, FMT>(p, d, smem, full, empty, ab, &uempty[us], &uent[us], hpub, hcount, gu, si, q, warp, lane);
       if (!ok) break;
     }
   }
   __syncthreads();
 }
 
+template <int FMT>
 static cudaError_t launch_decode(const DecodeParams& p, int grid, const CUtensorMap (&tmc)[3],
                                  const CUtensorMap (&tms)[3], const CUtensorMap& tm_x, const CUtensorMap& tm_h,
                                  cudaStream_t s) {
   ProfileScope prof(FT_KERNEL_FFN_DECODE, s);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(ffn_decode_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDecSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(ffn_decode_kernel, dim3(grid), dim3(kDecThreads), kDecSmemBytes, s, p, tmc[0], tms[0], tmc[1],
+  return launch_pdl(ffn_decode_kernel<FMT>, dim3(grid), dim3(kDecThreads), kDecSmemBytes, s, p, tmc[0], tms[0], tmc[1],
                     tms[1], tmc[2], tms[2], tm_x, tm_h);
 }
 

@@ -101,6 +101,26 @@ __device__ __forceinline__ uint32_t e4m3_pair_to_f16x2(uint32_t byte) {   // (s,
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(in));
   return r;
 }
+// E8M0 scale byte s of an MXFP4 block -> (2^(s - bias), 2^(s - bias)) in f16,
+// bias = 127 + t with 2^t the tensor's global: from the exponent bits (normal
+// for s - bias >= -14, subnormal down to 2^-24, zero below; the pack keeps
+// s - bias <= 13).
+__device__ __forceinline__ uint32_t e8m0_pair_to_f16x2(uint32_t byte, int bias) {
+  const int e = min(int(byte) - bias, 15);
+  const uint32_t h = e >= -14 ? uint32_t(e + 15) << 10 : (e >= -24 ? 1u << (e + 24) : 0u);
+  return h | (h << 16);
+}
+// The shift that the dequantisation takes out of MXFP4 scales: 127 + log2 of
+// the tensor's global (a power of two).
+__device__ __forceinline__ int mx_bias(float global) { return 127 + ilogbf(global); }
+
+// Scale byte of one 16-K block -> f16x2 (s, s) in the slot's format.
+template <int FMT>
+__device__ __forceinline__ uint32_t scale_pair_to_f16x2(uint32_t byte, int bias) {
+  if (FMT == FT_SCALE_MXFP4) return e8m0_pair_to_f16x2(byte, bias);
+  return e4m3_pair_to_f16x2(byte);
+}
+
 __device__ __forceinline__ uint32_t hmul2_f16(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -120,12 +140,13 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
 // f16x2 words, word c holding k = 2c (low half) and 2c + 1 (high half).
 // Every E2M1 x E4M3 product (at most 6 significant bits, magnitude in
 // [2^-10, 2688]) is an exact f16, so the products carry no rounding.
-__device__ __forceinline__ void dequant_chunk(const uint4& c0, const uint4& c1, uint32_t sc,
+template <int FMT>
+__device__ __forceinline__ void dequant_chunk(const uint4& c0, const uint4& c1, uint32_t sc, int bias,
                                               uint32_t (&o)[32]) {
   const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
-    const uint32_t s2 = e4m3_pair_to_f16x2((sc >> (8 * b)) & 0xFFu);
+    const uint32_t s2 = scale_pair_to_f16x2<FMT>((sc >> (8 * b)) & 0xFFu, bias);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t q[4];
@@ -194,7 +215,7 @@ __device__ __forceinline__ float token_factor(const FfnParams& p, int row) {
   return p.rowscale != nullptr ? __ldg(p.rowscale + row) : 1.0f;
 }
 
-template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC>
+template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
 ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0,
                 const __grid_constant__ CUtensorMap tm_scales0, const __grid_constant__ CUtensorMap tm_codes1,
@@ -398,6 +419,14 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       int e, mt, rb, nr, ws0, ws1, kc0, kc1;
       unit_range(u, e, mt, rb, nr, ws0, ws1, kc0, kc1);
+      int bias[NMAT];   // MXFP4: the power of two the unit's globals take out of the scales
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) bias[m] = 0;
+      if (FMT == FT_SCALE_MXFP4) {
+        const uint8_t* sbase = p.pool + size_t(__ldg(p.slot_table + e)) * size_t(p.slot_bytes);
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) bias[m] = mx_bias(__ldg(reinterpret_cast<const float*>(sbase + p.global_off[m])));
+      }
       for (int ws = ws0; ws < ws1 && ok; ++ws, ++wi) {
         const int s = wi % WS;
         if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&w_full[s], (wi / WS) & 1, kTagWFull, wi, u)))) break;
@@ -419,7 +448,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
               const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2 * t + 1) ^ (row & 7)) << 4));
               const uint32_t sc = *reinterpret_cast<const uint32_t*>(base + kCodesBytes + row * 16 + t * 4);
               uint32_t o[32];
-              dequant_chunk(c0, c1, sc, o);
+              dequant_chunk<FMT>(c0, c1, sc, bias[m], o);
               tmem_st_32x32b_x32(tmem + lane_base + Cfg::kDCols + (as * NMAT + m) * Cfg::kACols + h * 32, o);
             }
           }

@@ -186,13 +186,13 @@ static bool make_act_map(const void* base, int rows, int K, int box_rows, CUtens
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC>
+template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC, int FMT>
 static cudaError_t launch_gemm(const FfnParams& p, int grid, const CUtensorMap& c0, const CUtensorMap& s0,
                                const CUtensorMap& c1, const CUtensorMap& s1, const CUtensorMap& act,
                                cudaStream_t s) {
   ProfileScope prof(NMAT == 2 ? FT_KERNEL_GEMM_GATE_UP : FT_KERNEL_GEMM_DOWN, s);
   using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB, KC>;
-  auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB, KC>;
+  auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB, KC, FMT>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
@@ -317,11 +317,16 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
     dp.mt1 = pl.mt1;
     dp.mt2 = pl.mt2;
     const int grid = int(std::min<long long>(num_sms, pl.max_units1 + pl.max_units2));
-    err = launch_decode(dp, grid, tmc, tms, tm_x, tm_h, s);
-  } else {
-    err = launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    err = L.scale_format == FT_SCALE_MXFP4 ? launch_decode<FT_SCALE_MXFP4>(dp, grid, tmc, tms, tm_x, tm_h, s)
+                                           : launch_decode<FT_SCALE_NVFP4>(dp, grid, tmc, tms, tm_x, tm_h, s);
+  } else if (L.scale_format == FT_SCALE_MXFP4) {
+    err = launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1, FT_SCALE_MXFP4>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
     if (err == cudaSuccess)
-      err = launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
+      err = launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2, FT_SCALE_MXFP4>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
+  } else {
+    err = launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1, FT_SCALE_NVFP4>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    if (err == cudaSuccess)
+      err = launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2, FT_SCALE_NVFP4>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   }
   return err;
 }

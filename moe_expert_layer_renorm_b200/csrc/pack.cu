@@ -106,4 +106,73 @@ static cudaError_t launch_pack(const float* w, int N, int K, uint8_t* codes, uin
   return cudaGetLastError();
 }
 
+// MXFP4 (OCP Microscaling) pack: one E8M0 scale per 32 consecutive K of a
+// row, stored twice so that the slot layout matches NVFP4's one byte per 16:
+//   x_b = clamp(floor(log2 amax_b) - 2, -127, 127)   (-127 if amax_b = 0)
+//   q   = e2m1_rn_satfinite(w / 2^x_b)               (a power-of-two scaling: exact)
+// and the tensor's global = 2^t, t = clamp(floor(log2 amax) - 2) - 13, which
+// the GEMMs divide out of every dequantised f16 value (so e2m1 * 2^(x_b - t)
+// <= 6 * 2^13) and multiply back in fp32.  A block with x_b - t < -23 would
+// lose nonzero values to f16 underflow; it records FT_DEV_F16_RANGE.
+// One thread per scale byte position: even positions pack their 32-block.
+__global__ void __launch_bounds__(256) mxfp4_pack_kernel(const float* __restrict__ w, int N, int K,
+                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                         int ld_scale, const unsigned int* __restrict__ amax_bits,
+                                                         float* __restrict__ global_scale) {
+  const int nb16 = K / 16;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const float amax = __uint_as_float(*amax_bits);
+  const int t = amax > 0.0f ? max(-127, min(127, ilogbf(amax) - 2)) - 13 : 0;
+  if (i == 0) *global_scale = ldexpf(1.0f, t);
+  if (i >= (long long)N * ld_scale) return;
+  const int n = int(i / ld_scale), b16 = int(i % ld_scale);
+  if (b16 >= nb16) {  // scale-row padding
+    scales[size_t(n) * ld_scale + b16] = 0;
+    return;
+  }
+  if (b16 & 1) return;   // written by the even position of the pair
+  const int b = b16 / 2;
+  const float4* src = reinterpret_cast<const float4*>(w + size_t(n) * K + size_t(b) * 32);
+  float v[32];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 f = __ldg(src + q);
+    v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+  }
+  float amax_b = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) amax_b = fmaxf(amax_b, fabsf(v[q]));
+  const int x = amax_b > 0.0f ? max(-127, min(127, ilogbf(amax_b) - 2)) : -127;
+  if (amax_b > 0.0f && x - t < -23) set_device_status(FT_DEV_F16_RANGE);
+  uint32_t words[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const uint32_t byte = cvt_e2m1x2_satfinite(ldexpf(v[2 * q], -x), ldexpf(v[2 * q + 1], -x));
+    words[q / 4] |= byte << (8 * (q % 4));
+  }
+  uint2* dst = reinterpret_cast<uint2*>(codes + size_t(n) * (K / 2) + size_t(b) * 16);
+  dst[0] = make_uint2(words[0], words[1]);
+  dst[1] = make_uint2(words[2], words[3]);
+  scales[size_t(n) * ld_scale + 2 * b] = uint8_t(x + 127);
+  scales[size_t(n) * ld_scale + 2 * b + 1] = uint8_t(x + 127);
+}
+
+static cudaError_t launch_pack_mxfp4(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
+                                     float* global_scale, void* ws, cudaStream_t s) {
+  unsigned int* amax = static_cast<unsigned int*>(ws);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), s);
+  if (e != cudaSuccess) return e;
+  const long long n4 = (long long)N * K / 4;
+  const int blocks1 = int(std::min<long long>((n4 + 255) / 256, 148LL * 8));
+  {
+    ProfileScope prof(FT_KERNEL_PACK, s);
+    amax_kernel<<<blocks1, 256, 0, s>>>(reinterpret_cast<const float4*>(w), n4, amax);
+  }
+  const long long nthreads = (long long)N * ld_scale;
+  ProfileScope prof(FT_KERNEL_PACK, s);
+  mxfp4_pack_kernel<<<dim3(unsigned((nthreads + 255) / 256)), 256, 0, s>>>(w, N, K, codes, scales, ld_scale, amax,
+                                                                             global_scale);
+  return cudaGetLastError();
+}
+
 }  // namespace ftmoe

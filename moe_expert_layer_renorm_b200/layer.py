@@ -25,11 +25,12 @@ def _stream(s: Optional[torch.cuda.Stream]) -> int:
 
 
 class ExpertPool:
-    """A device pool of NVFP4 expert slots laid out by ft_nvfp4_slot_layout_init."""
+    """A device pool of expert slots (NVFP4, or MXFP4 with fmt=FT_SCALE_MXFP4)
+    laid out by ft_nvfp4_slot_layout_init / ft_mxfp4_slot_layout_init."""
 
-    def __init__(self, H: int, I: int, num_slots: int, device="cuda"):
-        self.H, self.I, self.num_slots = H, I, num_slots
-        self.layout = _lib.slot_layout(H, I, num_slots)
+    def __init__(self, H: int, I: int, num_slots: int, device="cuda", fmt: int = _lib.FT_SCALE_NVFP4):
+        self.H, self.I, self.num_slots, self.fmt = H, I, num_slots, fmt
+        self.layout = _lib.slot_layout(H, I, num_slots, fmt)
         self.slot_bytes = int(self.layout.slot_bytes)
         self.buf = torch.zeros(num_slots * self.slot_bytes, dtype=torch.uint8, device=device)
         self._pack_ws = torch.zeros(256, dtype=torch.uint8, device=device)
@@ -42,13 +43,14 @@ class ExpertPool:
         return (self.I, self.H) if mat in (FT_GATE, FT_UP) else (self.H, self.I)
 
     def pack_into(self, slot: int, mat: int, w: torch.Tensor, stream=None) -> None:
-        """Quantise fp32 weights w [N, K] (on the device) into `slot`."""
+        """Quantise fp32 weights w [N, K] (on the device) into `slot`, in the pool's format."""
         N, K = self.shape(mat)
         assert w.shape == (N, K) and w.dtype == torch.float32 and w.is_cuda and w.is_contiguous()
         L = self.layout
         base = self.ptr + slot * self.slot_bytes
-        _lib.nvfp4_pack(w.data_ptr(), N, K, base + L.codes_off[mat], base + L.scales_off[mat],
-                        L.ld_scale[mat], base + L.global_off[mat], self._pack_ws.data_ptr(), _stream(stream))
+        pack = _lib.mxfp4_pack if self.fmt == _lib.FT_SCALE_MXFP4 else _lib.nvfp4_pack
+        pack(w.data_ptr(), N, K, base + L.codes_off[mat], base + L.scales_off[mat], L.ld_scale[mat],
+             base + L.global_off[mat], self._pack_ws.data_ptr(), _stream(stream))
 
     def slot_view(self, slot: int) -> torch.Tensor:
         return self.buf[slot * self.slot_bytes:(slot + 1) * self.slot_bytes]

@@ -44,7 +44,7 @@ def lib() -> ctypes.CDLL:
         L.orc_moe_layer.argtypes = [POINTER(c_uint16), POINTER(c_float), c_int, c_int, c_int, c_int, c_int,
                                     POINTER(c_int32), POINTER(c_uint8), c_int64, POINTER(c_int64),
                                     POINTER(c_int64), POINTER(c_int64), POINTER(c_int32), POINTER(c_int32), c_int,
-                                    POINTER(c_double)]
+                                    c_int, POINTER(c_double)]
         _L = L
     return _L
 
@@ -125,8 +125,10 @@ def permute(ids: np.ndarray, E: int):
 
 def moe_layer(x_bits: np.ndarray, logits: np.ndarray, k: int, slot_table: np.ndarray, pool: np.ndarray,
               slot_bytes: int, codes_off: Sequence[int], scales_off: Sequence[int], global_off: Sequence[int],
-              ld_scale: Sequence[int], H: int, I: int, tokens: Optional[Sequence[int]] = None) -> np.ndarray:
-    """y fp64 [len(tokens), H] (all tokens by default) from a host copy of the slot pool."""
+              ld_scale: Sequence[int], H: int, I: int, tokens: Optional[Sequence[int]] = None,
+              fmt: int = 0) -> np.ndarray:
+    """y fp64 [len(tokens), H] (all tokens by default) from a host copy of the slot pool;
+    fmt 0: NVFP4 experts, 1: MXFP4 experts."""
     xb = np.ascontiguousarray(x_bits, dtype=np.uint16)
     lg = np.ascontiguousarray(logits, dtype=np.float32)
     T, E = lg.shape
@@ -140,7 +142,7 @@ def moe_layer(x_bits: np.ndarray, logits: np.ndarray, k: int, slot_table: np.nda
     y = np.zeros((len(tok), H), dtype=np.float64)
     rc = lib().orc_moe_layer(_p(xb, c_uint16), _p(lg, c_float), T, E, k, H, I, _p(st, c_int32), _p(pl, c_uint8),
                              slot_bytes, _p(co, c_int64), _p(so, c_int64), _p(go, c_int64), _p(ld, c_int32),
-                             _p(tok, c_int32), len(tok), _p(y, c_double))
+                             _p(tok, c_int32), len(tok), int(fmt), _p(y, c_double))
     if rc != 0:
         raise ValueError({-1: "bad argument", -2: "NaN scale byte", -3: "expert not resident"}.get(rc, str(rc)))
     return y

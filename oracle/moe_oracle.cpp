@@ -73,22 +73,31 @@ const Tables& tables() {
   return t;
 }
 
-// One NVFP4 tensor [N, K] as stored: codes [N, K/2] (even k in the low
-// nibble), scales [N, ld] bytes, one fp32 global scale.
+// One expert tensor [N, K] as stored in a slot: codes [N, K/2] (even k in
+// the low nibble), scales [N, ld] bytes, one fp32 global scale.
+//   NVFP4 (mx = false): e2m1(code) * e4m3(scale[k/16]) * global
+//   MXFP4 (mx = true):  e2m1(code) * e8m0(scale[k/16]); the slot stores each
+//                       32-block's E8M0 byte at both of its 16-K positions,
+//                       and the MX value has no global factor
 struct Tensor {
   const uint8_t* codes;
   const uint8_t* scales;
   double global;
   int N, K, ld;
+  bool mx;
+  double scale(int n, int k) const {
+    const uint8_t b = scales[size_t(n) * ld + k / 16];
+    return mx ? e8m0_value(b) : tables().e4m3[b] * global;
+  }
   double at(int n, int k) const {
     const uint8_t byte = codes[size_t(n) * (K / 2) + k / 2];
     const int code = (k & 1) ? (byte >> 4) : (byte & 15);
-    return tables().e2m1[code] * tables().e4m3[scales[size_t(n) * ld + k / 16]] * global;
+    return tables().e2m1[code] * scale(n, k);
   }
   bool has_nan_scale() const {
     for (int n = 0; n < N; ++n)
       for (int b = 0; b < K / 16; ++b)
-        if (std::isnan(tables().e4m3[scales[size_t(n) * ld + b]])) return true;
+        if (std::isnan(scale(n, 16 * b))) return true;
     return false;
   }
 };
@@ -269,13 +278,14 @@ int orc_permute(const int32_t* ids, int T, int k, int E, int32_t* offsets, int32
 //            pool + slot_table[e] * slot_bytes + codes_off[m], its scales at
 //            ... + scales_off[m] (ld_scale[m] bytes per row) and its fp32
 //            global scale at ... + global_off[m]
+//   fmt      0: NVFP4 experts; 1: MXFP4 experts (see Tensor)
 // Returns 0, -1 on a bad argument, -2 on a NaN scale byte, -3 on a
 // non-resident (slot < 0) expert.
 int orc_moe_layer(const uint16_t* x_bits, const float* logits, int T, int E, int k, int H, int I,
                   const int32_t* slot_table, const uint8_t* pool, int64_t slot_bytes, const int64_t* codes_off,
                   const int64_t* scales_off, const int64_t* global_off, const int32_t* ld_scale,
-                  const int32_t* tokens, int ntok, double* y) {
-  if (k < 1 || k > E || H % 16 || I % 16) return -1;
+                  const int32_t* tokens, int ntok, int fmt, double* y) {
+  if (k < 1 || k > E || H % 16 || I % 16 || (fmt != 0 && fmt != 1)) return -1;
   for (int i = 0; i < ntok; ++i)
     if (tokens[i] < 0 || tokens[i] >= T) return -1;
   int status = 0;
@@ -306,7 +316,7 @@ int orc_moe_layer(const uint16_t* x_bits, const float* logits, int T, int E, int
       for (int m = 0; m < 3; ++m) {
         float gs;
         std::memcpy(&gs, base + global_off[m], 4);
-        W[m] = Tensor{base + codes_off[m], base + scales_off[m], double(gs), rows[m], cols[m], ld_scale[m]};
+        W[m] = Tensor{base + codes_off[m], base + scales_off[m], double(gs), rows[m], cols[m], ld_scale[m], fmt == 1};
         if (W[m].has_nan_scale()) {
 #pragma omp atomic write
           status = -2;

@@ -14,10 +14,10 @@ from moe_expert_layer_renorm_b200.layer import ExpertPool, MoELayer
 from oracle import moe_layer as M
 
 
-def build_pool(w: inputs.Workload, layer: int = 0, device="cuda"):
+def build_pool(w: inputs.Workload, layer: int = 0, device="cuda", fmt: int = 0):
     s = inputs.layer_seed(w.seed, layer)
     slot_table = inputs.make_slot_table(w.E, w.slots, w.permuted_slots, s)
-    pool = ExpertPool(w.H, w.I, w.slots, device=device)
+    pool = ExpertPool(w.H, w.I, w.slots, device=device, fmt=fmt)
     for e in range(w.E):
         for mat in range(3):
             N, K = pool.shape(mat)
@@ -111,7 +111,8 @@ def reference_y(run: GpuRun, k: int, tok: np.ndarray) -> np.ndarray:
     buf, table, L = host_pool(run.pool, run.slot_table, ids[tok].reshape(-1))
     H, I = run.pool.H, run.pool.I
     return cpp.moe_layer(run.x_bits, run.logits, k, table, buf, run.pool.slot_bytes, list(L.codes_off),
-                         list(L.scales_off), list(L.global_off), list(L.ld_scale), H, I, tokens=tok)
+                         list(L.scales_off), list(L.global_off), list(L.ld_scale), H, I, tokens=tok,
+                         fmt=int(run.pool.layout.scale_format))
 
 
 def check_output(run: GpuRun, k: int, tokens: Optional[Sequence[int]] = None):

@@ -133,3 +133,48 @@ def test_numpy_and_cpp_oracles_agree_bit_for_bit():
     c2, s2 = mxfp4.pack(w)
     assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
     assert np.array_equal(cpp.decode_mxfp4(c1, s1, 128), mxfp4.decode(c2, s2, 128))
+
+
+def test_layer_with_mxfp4_experts_is_the_dense_layer():
+    """The oracle's layer over MXFP4 experts read from a slot pool (each E8M0
+    byte stored at both of its 16-K positions, the global ignored) equals the
+    same layer computed densely from decode_mxfp4 of each tensor."""
+    import bench
+    from moe_expert_layer_renorm_b200 import inputs
+    w = inputs.WORKLOADS["tiny"]
+    L = bench.reference_layout(w.H, w.I)
+    s = inputs.layer_seed(w.seed, 0)
+    st = np.arange(w.E, dtype=np.int32)
+    pool = np.zeros(w.E * L["slot_bytes"], np.uint8)
+    dense = {}
+    shapes = [(w.I, w.H), (w.I, w.H), (w.H, w.I)]
+    for e in range(w.E):
+        base = e * L["slot_bytes"]
+        mats = []
+        for m, (N, K) in enumerate(shapes):
+            wt = inputs.make_weight_fp32_host(N, K, s, e, m)
+            codes, sc = cpp.pack_mxfp4(wt)
+            mats.append(cpp.decode_mxfp4(codes, sc, K))
+            ld = L["ld_scale"][m]
+            sc16 = np.zeros((N, ld), np.uint8)
+            sc16[:, 0:K // 16:2] = sc
+            sc16[:, 1:K // 16:2] = sc
+            o = base + L["codes_off"][m]
+            pool[o:o + codes.size] = codes.reshape(-1)
+            o = base + L["scales_off"][m]
+            pool[o:o + sc16.size] = sc16.reshape(-1)
+            o = base + L["global_off"][m]
+            pool[o:o + 4] = np.frombuffer(np.float32(1024.0).tobytes(), np.uint8)   # must not matter
+        dense[e] = mats
+    li = inputs.make_layer_inputs(w)
+    y = cpp.moe_layer(li.x_bits, li.logits, w.k, st, pool, L["slot_bytes"], L["codes_off"], L["scales_off"],
+                      L["global_off"], L["ld_scale"], w.H, w.I, fmt=1)
+    ids, wts = cpp.route(li.logits, w.k)
+    x = inputs.bf16_bits_to_fp32(li.x_bits).astype(np.float64)
+    ref = np.zeros_like(y)
+    for t in range(x.shape[0]):
+        for j in range(w.k):
+            g_, u_, d_ = dense[int(ids[t, j])]
+            G, U = g_ @ x[t], u_ @ x[t]
+            ref[t] += wts[t, j] * (d_ @ (G * U / (1.0 + np.exp(-G))))
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
