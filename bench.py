@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"], help="expert weight format")
+    ap.add_argument("--fused-front", action="store_true",
+                    help="route and permute through ft_moe_route_permute (one launch for small batches)")
     ap.add_argument("--slot-churn", nargs="?", const="decode", default=None, choices=["decode", "prefill_stream"],
                     help="measure the expert-cache miss path (pinned host banks, LRU slot manager) instead: "
                          "domain-rotation decode steps, or prefill layers streamed through a two-layer pool")
@@ -295,7 +297,7 @@ def run_ours(args):
         lg = torch.from_numpy(li.logits).to(dev)
         layers.append(dict(li=li, pool=pool, st_host=st, st=torch.from_numpy(st).to(dev), x=x, lg=lg, seed=s))
     torch.cuda.synchronize()
-    layer = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev)
+    layer = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev, fused_front=args.fused_front)
     stream = torch.cuda.Stream(device=dev)
 
     # distinct experts per layer (routing is deterministic; used for the algorithmic bytes)
@@ -367,7 +369,8 @@ def run_ours(args):
         host.append((L["x"].cpu().pin_memory(), L["lg"].cpu().pin_memory()))
     bufs = []
     for _ in range(2):
-        bufs.append(dict(lay=MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev),
+        bufs.append(dict(lay=MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev,
+                                      fused_front=args.fused_front),
                          xd=torch.empty_like(layers[0]["x"]), lgd=torch.empty_like(layers[0]["lg"]),
                          y_host=torch.empty((T, w.H), dtype=torch.float32).pin_memory()))
     e2e_graphs = {}
@@ -495,7 +498,8 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": f"{args.fmt} weights, f16 MMA operands, fp32 accumulate",
         "data": "synthetic (seeded N(0,1) activations, N(0,sigma) logits, N(0,0.02) weights packed to NVFP4)",
-        "config": dict(workload_config(w, R, S, world, mean_distinct), format=args.fmt),
+        "config": dict(workload_config(w, R, S, world, mean_distinct), format=args.fmt,
+                       front="ft_moe_route_permute" if args.fused_front else "ft_moe_route + ft_moe_permute"),
         "layer": {"distinct_experts": round(mean_distinct, 2), "weight_GBps": round(layer_gbs, 1),
                   "TFLOPs": round(layer_tflops, 2), "hbm_frac_of_measured": round(layer_gbs / hbm, 4)},
         "roofline": roof,
