@@ -108,3 +108,30 @@ def test_reference_layout_matches_library(H, I):
     assert list(L.ld_scale) == ref["ld_scale"] and list(L.codes_off) == ref["codes_off"]
     assert list(L.scales_off) == ref["scales_off"] and list(L.global_off) == ref["global_off"]
     assert L.slot_bytes == ref["slot_bytes"]
+
+
+def test_argument_checks_of_the_later_entry_points(L):
+    # route + permute in one call: the route rules, and T == 0 needs offsets only
+    assert L.ft_moe_route_permute(None, 4, 8, 9, 0, None, None, None, None, None, None, 0, None) \
+        == _lib.FT_ERR_INVALID_ARG
+    assert L.ft_moe_route_permute(None, 4, 8, 2, 2, None, None, None, None, None, None, 0, None) \
+        == _lib.FT_ERR_INVALID_ARG                                       # mode 2
+    assert L.ft_moe_route_permute(None, 0, 8, 2, 0, None, None, None, None, None, None, 0, None) \
+        == _lib.FT_ERR_INVALID_ARG                                       # no offsets to clear
+    assert b"null" in L.ft_last_error()
+    # row gather: row length a positive multiple of 16 bytes, div >= 1; n == 0 is a no-op
+    assert L.ft_gather_rows(None, 4, 24, None, 1, 4, None, None) == _lib.FT_ERR_INVALID_ARG
+    assert L.ft_gather_rows(None, 4, 32, None, 0, 4, None, None) == _lib.FT_ERR_INVALID_ARG
+    assert L.ft_gather_rows(None, 4, 32, None, 1, 4, None, None) == _lib.FT_ERR_INVALID_ARG   # null pointers
+    assert L.ft_gather_rows(None, 4, 32, None, 1, 0, None, None) == _lib.FT_OK
+    assert L.ft_selftest_wait_timeout(None, None) == _lib.FT_ERR_INVALID_ARG
+    # MXFP4 pack: K a multiple of 32
+    assert L.ft_mxfp4_pack(None, 4, 48, None, None, 16, None, None, None) == _lib.FT_ERR_INVALID_ARG
+
+
+def test_mxfp4_layout_is_the_nvfp4_layout_with_its_tag(L):
+    a, b = _lib.slot_layout(2048, 768, 5), _lib.slot_layout(2048, 768, 5, _lib.FT_SCALE_MXFP4)
+    assert (a.scale_format, b.scale_format) == (_lib.FT_SCALE_NVFP4, _lib.FT_SCALE_MXFP4)
+    for f in ("ld_scale", "codes_off", "scales_off", "global_off"):
+        assert list(getattr(a, f)) == list(getattr(b, f))
+    assert a.slot_bytes == b.slot_bytes
