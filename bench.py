@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"], help="expert weight format")
+    ap.add_argument("--layout", default="rows", choices=["rows", "tiled"],
+                    help="expert slot layout: row-major tensors, or stage-tiled (each weight box contiguous)")
     ap.add_argument("--fused-front", action="store_true",
                     help="route and permute through ft_moe_route_permute (one launch for small batches)")
     ap.add_argument("--slot-churn", nargs="?", const="decode", default=None, choices=["decode", "prefill_stream"],
@@ -260,6 +262,12 @@ class E2EPipeline:
         self.compute.wait_event(self.out_done[(n - 1) % self.nbuf])
 
 
+def run_config(args, base: dict) -> dict:
+    """The reported config: the workload's, plus the options that change what runs."""
+    return dict(base, format=args.fmt, slot_layout=args.layout,
+                front="ft_moe_route_permute" if args.fused_front else "ft_moe_route + ft_moe_permute")
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -283,7 +291,8 @@ def run_ours(args):
     S = max(w.slots, R * w.E)
     order = np.random.default_rng([w.seed, rank, 9]).permutation(S) if w.permuted_slots else np.arange(S)
     pool = ExpertPool(w.H, w.I, S, device=dev,
-                      fmt=_lib.FT_SCALE_MXFP4 if args.fmt == "mxfp4" else _lib.FT_SCALE_NVFP4)
+                      fmt=_lib.FT_SCALE_MXFP4 if args.fmt == "mxfp4" else _lib.FT_SCALE_NVFP4,
+                      tiled=args.layout == "tiled")
     layers = []
     for l in range(R):
         s = rank_layer_seed(w, rank, l)
@@ -498,8 +507,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": f"{args.fmt} weights, f16 MMA operands, fp32 accumulate",
         "data": "synthetic (seeded N(0,1) activations, N(0,sigma) logits, N(0,0.02) weights packed to NVFP4)",
-        "config": dict(workload_config(w, R, S, world, mean_distinct), format=args.fmt,
-                       front="ft_moe_route_permute" if args.fused_front else "ft_moe_route + ft_moe_permute"),
+        "config": run_config(args, workload_config(w, R, S, world, mean_distinct)),
         "layer": {"distinct_experts": round(mean_distinct, 2), "weight_GBps": round(layer_gbs, 1),
                   "TFLOPs": round(layer_tflops, 2), "hbm_frac_of_measured": round(layer_gbs / hbm, 4)},
         "roofline": roof,
@@ -534,16 +542,17 @@ def cpu_baseline(L, w, T, n_tokens, fmt="nvfp4"):
     n = min(T, n_tokens)
     ids, _ = cpp.route(li.logits[:n], w.k)
     need = sorted(set(int(v) for v in ids.reshape(-1)))
-    buf = np.zeros(len(need) * pool.slot_bytes, np.uint8)     # the selected experts' slots, on the host
+    Lo = pool.rows_layout                                     # slots read back row-major
+    nb = int(Lo.slot_bytes)
+    buf = np.zeros(len(need) * nb, np.uint8)                  # the selected experts' slots, on the host
     table = np.full(w.E, -1, np.int32)
     for i, e in enumerate(need):
-        buf[i * pool.slot_bytes:(i + 1) * pool.slot_bytes] = pool.slot_view(int(st[e])).cpu().numpy()
+        buf[i * nb:(i + 1) * nb] = pool.export_slot(int(st[e]))
         table[e] = i
-    Lo = pool.layout
     reps, dt = 0, 0.0
     while dt < 10.0 and reps < 50:
         t0 = time.perf_counter()
-        cpp.moe_layer(li.x_bits, li.logits, w.k, table, buf, pool.slot_bytes, list(Lo.codes_off),
+        cpp.moe_layer(li.x_bits, li.logits, w.k, table, buf, nb, list(Lo.codes_off),
                       list(Lo.scales_off), list(Lo.global_off), list(Lo.ld_scale), w.H, w.I, tokens=np.arange(n),
                       fmt=int(Lo.scale_format))
         dt += time.perf_counter() - t0
@@ -639,7 +648,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": dict(format=args.fmt, **workload_config(
+        "data": "synthetic", "config": run_config(args, workload_config(
             w, R, max(w.slots, R * w.E), world, inputs.expected_distinct_experts(w.T, w.E, w.k))),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": f"{n} tokens of one {w.name} layer per step"},

@@ -100,6 +100,8 @@ typedef struct {
   int64_t slot_bytes;
   int32_t num_slots;      /* slots in the pool the layout describes */
   int32_t scale_format;   /* FT_SCALE_NVFP4 or FT_SCALE_MXFP4 */
+  int32_t tiled;          /* 0: codes [N, K/2] and scales [N, ld_scale] row-major;
+                             1: stage-tiled (see ft_tiled_slot_layout_init) */
 } ft_nvfp4_slot_layout;
 
 /* How a slot's scale bytes and global scales read.
@@ -120,6 +122,28 @@ enum { FT_SCALE_NVFP4 = 0, FT_SCALE_MXFP4 = 1 };
 FT_API int ft_nvfp4_slot_layout_init(int H, int I, int num_slots, ft_nvfp4_slot_layout* out);
 /* The same layout with scale_format = FT_SCALE_MXFP4 (identical offsets). */
 FT_API int ft_mxfp4_slot_layout_init(int H, int I, int num_slots, ft_nvfp4_slot_layout* out);
+/*
+ * A stage-tiled slot layout (tiled = 1) in either scale format.  The same
+ * bytes are arranged so that what the expert GEMMs load together is
+ * contiguous: for a tensor [N, K] with S = ceil(K / 256) stages of 256 K,
+ *   codes   uint8 [S][N][128]  byte (s, n, j) holds k = 256 s + 2 j, 2 j + 1
+ *   scales  uint8 [S][N][16]   byte (s, n, j) is the scale of k / 16 = 16 s + j
+ * so one stage of 128 rows is one 16 KB block of codes and one 2 KB block of
+ * scales.  Bytes past K/2 in the last stage hold zero codes.  ld_scale
+ * (= 16 S) and the global offsets keep their meaning.
+ */
+FT_API int ft_tiled_slot_layout_init(int H, int I, int num_slots, int scale_format,
+                                     ft_nvfp4_slot_layout* out);
+
+/*
+ * Pack fp32 weights w [N, K] (device; N, K the shape of tensor `mat` of the
+ * layout) into the tensor's place in one slot (slot: device address of the
+ * slot's first byte), in the layout's scale format and arrangement: the
+ * arithmetic of ft_nvfp4_pack or ft_mxfp4_pack, the bytes placed as the
+ * layout says.  ws as for those calls.
+ */
+FT_API int ft_pack_slot(const float* w, int mat, const ft_nvfp4_slot_layout* layout, void* slot, void* ws,
+                        ft_stream_t stream);
 
 /*
  * Router: per token t, the k experts with the largest logits (descending;

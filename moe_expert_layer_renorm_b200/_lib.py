@@ -49,6 +49,7 @@ class SlotLayout(ctypes.Structure):
         ("slot_bytes", c_int64),
         ("num_slots", c_int32),
         ("scale_format", c_int32),
+        ("tiled", c_int32),
     ]
 
 
@@ -68,6 +69,8 @@ class SlotStats(ctypes.Structure):
 _SIGS = {
     "ft_nvfp4_slot_layout_init": (c_int, [c_int, c_int, c_int, POINTER(SlotLayout)]),
     "ft_mxfp4_slot_layout_init": (c_int, [c_int, c_int, c_int, POINTER(SlotLayout)]),
+    "ft_tiled_slot_layout_init": (c_int, [c_int, c_int, c_int, c_int, POINTER(SlotLayout)]),
+    "ft_pack_slot": (c_int, [c_void_p, c_int, POINTER(SlotLayout), c_void_p, c_void_p, c_void_p]),
     "ft_moe_route": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "ft_moe_permute": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                c_void_p]),
@@ -125,11 +128,18 @@ def check(code: int) -> None:
 FT_SCALE_NVFP4, FT_SCALE_MXFP4 = 0, 1
 
 
-def slot_layout(H: int, I: int, num_slots: int, fmt: int = FT_SCALE_NVFP4) -> SlotLayout:
+def slot_layout(H: int, I: int, num_slots: int, fmt: int = FT_SCALE_NVFP4, tiled: bool = False) -> SlotLayout:
     L = SlotLayout()
+    if tiled:
+        check(lib().ft_tiled_slot_layout_init(H, I, num_slots, fmt, ctypes.byref(L)))
+        return L
     init = lib().ft_mxfp4_slot_layout_init if fmt == FT_SCALE_MXFP4 else lib().ft_nvfp4_slot_layout_init
     check(init(H, I, num_slots, ctypes.byref(L)))
     return L
+
+
+def pack_slot(w, mat, layout: SlotLayout, slot, ws, stream) -> None:
+    check(lib().ft_pack_slot(w, mat, ctypes.byref(layout), slot, ws, stream))
 
 
 def route(logits, T, E, k, mode, ids, w, stream) -> None:

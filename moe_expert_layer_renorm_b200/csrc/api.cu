@@ -67,6 +67,40 @@ extern "C" int ft_mxfp4_slot_layout_init(int H, int I, int num_slots, ft_nvfp4_s
   return rc;
 }
 
+extern "C" int ft_tiled_slot_layout_init(int H, int I, int num_slots, int scale_format, ft_nvfp4_slot_layout* out) {
+  if (!out || H <= 0 || I <= 0 || H % 64 || I % 64 || num_slots <= 0 ||
+      (scale_format != FT_SCALE_NVFP4 && scale_format != FT_SCALE_MXFP4))
+    return fail(FT_ERR_INVALID_ARG, "ft_tiled_slot_layout_init: need H, I multiples of 64, num_slots > 0, a format");
+  ft_nvfp4_slot_layout L{};
+  L.H = H;
+  L.I = I;
+  L.num_slots = num_slots;
+  const int rows[3] = {I, I, H}, Ks[3] = {H, H, I};
+  auto a256 = [](long long v) { return (v + 255) & ~255LL; };
+  long long off = 0;
+  for (int m = 0; m < 3; ++m) {
+    const long long stages = (Ks[m] + 255) / 256;
+    L.ld_scale[m] = int(16 * stages);
+    L.codes_off[m] = off;
+    off = a256(off + stages * rows[m] * 128);
+    L.scales_off[m] = off;
+    off = a256(off + stages * rows[m] * 16);
+  }
+  for (int m = 0; m < 3; ++m) L.global_off[m] = off + 4 * m;
+  off = a256(off + 12);
+  L.slot_bytes = off;
+  L.scale_format = scale_format;
+  L.tiled = 1;
+  *out = L;
+  return FT_OK;
+}
+
+static bool layout_ok(const ft_nvfp4_slot_layout* L) {
+  return L && L->H > 0 && L->I > 0 && L->H % 64 == 0 && L->I % 64 == 0 && L->num_slots >= 1 &&
+         L->slot_bytes % 256 == 0 && (L->tiled == 0 || L->tiled == 1) &&
+         (L->scale_format == FT_SCALE_NVFP4 || L->scale_format == FT_SCALE_MXFP4);
+}
+
 extern "C" int ft_moe_route(const float* logits, int T, int E, int k, int mode, int32_t* ids, float* w,
                             ft_stream_t stream) {
   if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32 || (mode != 0 && mode != 1))
@@ -141,6 +175,7 @@ extern "C" int ft_moe_ffn_nvfp4(const void* x, int T, int H, int I, int E, int k
   if (!x || !perm_src || !expert_offsets || !slot_table || !slot_pool || !layout || !out_perm || !ws)
     return fail(FT_ERR_INVALID_ARG, "ft_moe_ffn_nvfp4: null pointer");
   if (layout->H != H || layout->I != I || layout->num_slots < 1 || layout->num_slots > (1 << 21) ||
+      (layout->tiled != 0 && layout->tiled != 1) ||
       layout->slot_bytes % 256 ||
       (layout->scale_format != FT_SCALE_NVFP4 && layout->scale_format != FT_SCALE_MXFP4))
     return fail(FT_ERR_INVALID_ARG,
@@ -187,8 +222,33 @@ extern "C" int ft_nvfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8
   if (!w || !codes || !scales || !global_scale || !ws) return fail(FT_ERR_INVALID_ARG, "ft_nvfp4_pack: null pointer");
   if ((reinterpret_cast<uintptr_t>(w) & 15) || (reinterpret_cast<uintptr_t>(codes) & 7) || ((K / 2) % 8))
     return fail(FT_ERR_INVALID_ARG, "ft_nvfp4_pack: w must be 16-byte and codes 8-byte aligned");
-  const cudaError_t e = launch_pack(w, N, K, codes, scales, ld_scale, global_scale, ws, S(stream));
+  const cudaError_t e =
+      launch_pack(w, N, K, row_major_place(codes, scales, K, ld_scale), ld_scale, global_scale, ws, S(stream));
   return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_nvfp4_pack");
+}
+
+extern "C" int ft_pack_slot(const float* w, int mat, const ft_nvfp4_slot_layout* L, void* slot, void* ws,
+                            ft_stream_t stream) {
+  if (!layout_ok(L) || mat < 0 || mat > 2)
+    return fail(FT_ERR_INVALID_ARG, "ft_pack_slot: bad layout or tensor index");
+  if (!w || !slot || !ws) return fail(FT_ERR_INVALID_ARG, "ft_pack_slot: null pointer");
+  if ((reinterpret_cast<uintptr_t>(w) & 15) || (reinterpret_cast<uintptr_t>(slot) & 255))
+    return fail(FT_ERR_INVALID_ARG, "ft_pack_slot: w must be 16-byte and the slot 256-byte aligned");
+  const int N = mat == FT_DOWN ? L->H : L->I, K = mat == FT_DOWN ? L->I : L->H;
+  uint8_t* base = static_cast<uint8_t*>(slot);
+  PackPlace pl;
+  pl.codes = base + L->codes_off[mat];
+  pl.scales = base + L->scales_off[mat];
+  pl.tiled = L->tiled;
+  pl.c_row = L->tiled ? 128 : K / 2;
+  pl.c_stage = L->tiled ? 128LL * N : 128;
+  pl.s_row = L->tiled ? 16 : L->ld_scale[mat];
+  pl.s_stage = L->tiled ? 16LL * N : 16;
+  float* g = reinterpret_cast<float*>(base + L->global_off[mat]);
+  const cudaError_t e = L->scale_format == FT_SCALE_MXFP4
+                            ? launch_pack_mxfp4(w, N, K, pl, L->ld_scale[mat], g, ws, S(stream))
+                            : launch_pack(w, N, K, pl, L->ld_scale[mat], g, ws, S(stream));
+  return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_pack_slot");
 }
 
 extern "C" int ft_mxfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
@@ -198,7 +258,8 @@ extern "C" int ft_mxfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8
   if (!w || !codes || !scales || !global_scale || !ws) return fail(FT_ERR_INVALID_ARG, "ft_mxfp4_pack: null pointer");
   if ((reinterpret_cast<uintptr_t>(w) & 15) || (reinterpret_cast<uintptr_t>(codes) & 7) || ((K / 2) % 8))
     return fail(FT_ERR_INVALID_ARG, "ft_mxfp4_pack: w must be 16-byte and codes 8-byte aligned");
-  const cudaError_t e = launch_pack_mxfp4(w, N, K, codes, scales, ld_scale, global_scale, ws, S(stream));
+  const cudaError_t e = launch_pack_mxfp4(w, N, K, row_major_place(codes, scales, K, ld_scale), ld_scale,
+                                          global_scale, ws, S(stream));
   return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_mxfp4_pack");
 }
 

@@ -434,10 +434,11 @@ ffn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_c
             uent[us] = make_int4(q, __float_as_int(c.g0), __float_as_int(c.g1), 0);
           mbar_arrive_expect_tx(&full[s], kDecWStageBytes);
           uint8_t* st = smem + s * kDecStageBytes;
-          tma_load_3d(st, c0, &full[s], ws * 128, y0, slot);
-          tma_load_3d(st + 128 * 128, c1, &full[s], ws * 128, y1, slot);
-          tma_load_3d(st + kDecCodes, s0, &full[s], ws * 16, y0, slot);
-          tma_load_3d(st + kDecCodes + 128 * 16, s1, &full[s], ws * 16, y1, slot);
+          const int tl = p.g[0].tiled;
+          tma_load_weights(st, c0, &full[s], tl, 128, ws, y0, slot);
+          tma_load_weights(st + 128 * 128, c1, &full[s], tl, 128, ws, y1, slot);
+          tma_load_weights(st + kDecCodes, s0, &full[s], tl, 16, ws, y0, slot);
+          tma_load_weights(st + kDecCodes + 128 * 16, s1, &full[s], tl, 16, ws, y1, slot);
         }
         next_raw = next_q < ntot ? unit_desc(p, next_q, n1) : make_int4(0, 0, 0, 0);
       }

@@ -63,6 +63,7 @@ struct FfnParams {
   void* out;                  // GEMM1: h f16 [P, M]; GEMM2: out_perm fp32 [P, M]
   float* partials;            // split-K partial accumulators
   int* counters;              // split-K arrival counters, 4 per (tile, m_tile): one per epilogue warp
+  int tiled;                  // weight maps are 4-D over stage-tiled slots (else 3-D over row-major ones)
 };
 
 // KC: K per chunk (64 or 128), the unit of one dequantised A slot, one
@@ -293,8 +294,8 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
             uint8_t* dst = w_smem + (s * NMAT + m) * kMatStageBytes;
-            tma_load_3d(dst, tmc[m], &w_full[s], ws * 128, mt * 128, slot);
-            tma_load_3d(dst + kCodesBytes, tms[m], &w_full[s], ws * 16, mt * 128, slot);
+            tma_load_weights(dst, tmc[m], &w_full[s], p.tiled, 128, ws, mt * 128, slot);
+            tma_load_weights(dst + kCodesBytes, tms[m], &w_full[s], p.tiled, 16, ws, mt * 128, slot);
           }
         }
       }

@@ -145,10 +145,36 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // codes: [rows, K/2] bytes per slot, 128 x 128-byte boxes, 128-byte swizzle.
 // scales: [rows, ld_scale] bytes per slot, 128 x 16-byte boxes.
+// Stage-tiled slots: codes [S][rows][128] and scales [S][rows][16] per slot,
+// 4-D maps (bytes, rows, stage, slot) with the same boxes, so that a box is
+// one contiguous block of memory.
 static bool make_weight_maps(const uint8_t* pool, const ft_nvfp4_slot_layout& L, int mat, int rows, int K,
                              int box_rows, CUtensorMap* codes, CUtensorMap* scales) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
+  if (L.tiled) {
+    const cuuint64_t stages = cuuint64_t((K + 255) / 256);
+    const cuuint32_t es4[4] = {1, 1, 1, 1};
+    {
+      const cuuint64_t dims[4] = {128, cuuint64_t(rows), stages, cuuint64_t(L.num_slots)};
+      const cuuint64_t strides[3] = {128, cuuint64_t(rows) * 128, cuuint64_t(L.slot_bytes)};
+      const cuuint32_t box[4] = {128, cuuint32_t(box_rows), 1, 1};
+      if (enc(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, (void*)(pool + L.codes_off[mat]), dims, strides, box, es4,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    }
+    {
+      const cuuint64_t dims[4] = {16, cuuint64_t(rows), stages, cuuint64_t(L.num_slots)};
+      const cuuint64_t strides[3] = {16, cuuint64_t(rows) * 16, cuuint64_t(L.slot_bytes)};
+      const cuuint32_t box[4] = {16, cuuint32_t(box_rows), 1, 1};
+      if (enc(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, (void*)(pool + L.scales_off[mat]), dims, strides, box, es4,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    }
+    return true;
+  }
   const cuuint32_t elem_strides[3] = {1, 1, 1};
   {
     const cuuint64_t dims[3] = {cuuint64_t(K / 2), cuuint64_t(rows), cuuint64_t(L.num_slots)};
@@ -288,6 +314,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   p1.out = h;
   p1.partials = reinterpret_cast<float*>(w + pl.off_part1);
   p1.counters = cnt1;
+  p1.tiled = L.tiled;
   const int grid1 = int(std::min<long long>(num_sms, pl.max_units1));
 
   FfnParams p2 = p1;

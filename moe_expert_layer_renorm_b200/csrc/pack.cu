@@ -11,6 +11,37 @@
 
 namespace ftmoe {
 
+// Where a packed tensor's bytes go.  Code byte j of row n (codes of k = 2j,
+// 2j + 1) lives at codes + (j / 128) * c_stage + n * c_row + j % 128 and
+// scale byte b at scales + (b / 16) * s_stage + n * s_row + b % 16: row-major
+// [N, K/2] and [N, ld] with (c_row, c_stage, s_row, s_stage) = (K/2, 128,
+// ld, 16); stage-tiled [S][N][128] and [S][N][16] with (128, 128 N, 16, 16 N).
+// A tiled tensor also gets zero code bytes past K/2 in its last stage.
+struct PackPlace {
+  uint8_t* codes;
+  uint8_t* scales;
+  int tiled;
+  long long c_row, c_stage, s_row, s_stage;
+  __host__ __device__ uint8_t* code_at(int n, long long j) const {
+    return codes + (j / 128) * c_stage + n * c_row + (j % 128);
+  }
+  __host__ __device__ uint8_t* scale_at(int n, long long b) const {
+    return scales + (b / 16) * s_stage + n * s_row + (b % 16);
+  }
+};
+
+static PackPlace row_major_place(uint8_t* codes, uint8_t* scales, int K, int ld_scale) {
+  PackPlace p;
+  p.codes = codes;
+  p.scales = scales;
+  p.tiled = 0;
+  p.c_row = K / 2;
+  p.c_stage = 128;
+  p.s_row = ld_scale;
+  p.s_stage = 16;
+  return p;
+}
+
 __global__ void __launch_bounds__(256) amax_kernel(const float4* __restrict__ w, long long n4,
                                                    unsigned int* __restrict__ amax_bits) {
   float m = 0.0f;
@@ -46,8 +77,7 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2_satfinite(float lo, float hi) {
 }
 
 // One thread per 16-element block.
-__global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ w, int N, int K,
-                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+__global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ w, int N, int K, const PackPlace pl,
                                                    int ld_scale, const unsigned int* __restrict__ amax_bits,
                                                    float* __restrict__ global_scale) {
   const int nb = K / 16;
@@ -57,8 +87,9 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ w, 
   if (i == 0) *global_scale = g;
   if (i >= (long long)N * ld_scale) return;
   const int n = int(i / ld_scale), b = int(i % ld_scale);
-  if (b >= nb) {  // scale-row padding
-    scales[size_t(n) * ld_scale + b] = 0;
+  if (b >= nb) {  // scale-row padding (and, tiled, the code bytes of the same K range)
+    *pl.scale_at(n, b) = 0;
+    if (pl.tiled) *reinterpret_cast<uint2*>(pl.code_at(n, 8LL * b)) = make_uint2(0u, 0u);
     return;
   }
   const float4* src = reinterpret_cast<const float4*>(w + size_t(n) * K + size_t(b) * 16);
@@ -83,12 +114,11 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ w, 
       words[q / 4] |= byte << (8 * (q % 4));
     }
   }
-  uint2* dst = reinterpret_cast<uint2*>(codes + size_t(n) * (K / 2) + size_t(b) * 8);
-  *dst = make_uint2(words[0], words[1]);
-  scales[size_t(n) * ld_scale + b] = uint8_t(sbyte);
+  *reinterpret_cast<uint2*>(pl.code_at(n, 8LL * b)) = make_uint2(words[0], words[1]);
+  *pl.scale_at(n, b) = uint8_t(sbyte);
 }
 
-static cudaError_t launch_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
+static cudaError_t launch_pack(const float* w, int N, int K, const PackPlace& pl, int ld_scale,
                                float* global_scale, void* ws, cudaStream_t s) {
   unsigned int* amax = static_cast<unsigned int*>(ws);
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), s);
@@ -101,8 +131,7 @@ static cudaError_t launch_pack(const float* w, int N, int K, uint8_t* codes, uin
   }
   const long long nthreads = (long long)N * ld_scale;
   ProfileScope prof(FT_KERNEL_PACK, s);
-  pack_kernel<<<dim3(unsigned((nthreads + 255) / 256)), 256, 0, s>>>(w, N, K, codes, scales, ld_scale, amax,
-                                                                       global_scale);
+  pack_kernel<<<dim3(unsigned((nthreads + 255) / 256)), 256, 0, s>>>(w, N, K, pl, ld_scale, amax, global_scale);
   return cudaGetLastError();
 }
 
@@ -116,8 +145,8 @@ static cudaError_t launch_pack(const float* w, int N, int K, uint8_t* codes, uin
 // lose nonzero values to f16 underflow; it records FT_DEV_F16_RANGE.
 // One thread per scale byte position: even positions pack their 32-block.
 __global__ void __launch_bounds__(256) mxfp4_pack_kernel(const float* __restrict__ w, int N, int K,
-                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                                         int ld_scale, const unsigned int* __restrict__ amax_bits,
+                                                         const PackPlace pl, int ld_scale,
+                                                         const unsigned int* __restrict__ amax_bits,
                                                          float* __restrict__ global_scale) {
   const int nb16 = K / 16;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -126,8 +155,9 @@ __global__ void __launch_bounds__(256) mxfp4_pack_kernel(const float* __restrict
   if (i == 0) *global_scale = ldexpf(1.0f, t);
   if (i >= (long long)N * ld_scale) return;
   const int n = int(i / ld_scale), b16 = int(i % ld_scale);
-  if (b16 >= nb16) {  // scale-row padding
-    scales[size_t(n) * ld_scale + b16] = 0;
+  if (b16 >= nb16) {  // scale-row padding (and, tiled, the code bytes of the same K range)
+    *pl.scale_at(n, b16) = 0;
+    if (pl.tiled) *reinterpret_cast<uint2*>(pl.code_at(n, 8LL * b16)) = make_uint2(0u, 0u);
     return;
   }
   if (b16 & 1) return;   // written by the even position of the pair
@@ -150,14 +180,14 @@ __global__ void __launch_bounds__(256) mxfp4_pack_kernel(const float* __restrict
     const uint32_t byte = cvt_e2m1x2_satfinite(ldexpf(v[2 * q], -x), ldexpf(v[2 * q + 1], -x));
     words[q / 4] |= byte << (8 * (q % 4));
   }
-  uint2* dst = reinterpret_cast<uint2*>(codes + size_t(n) * (K / 2) + size_t(b) * 16);
+  uint2* dst = reinterpret_cast<uint2*>(pl.code_at(n, 16LL * b));   // 16 bytes inside one 128-byte stage row
   dst[0] = make_uint2(words[0], words[1]);
   dst[1] = make_uint2(words[2], words[3]);
-  scales[size_t(n) * ld_scale + 2 * b] = uint8_t(x + 127);
-  scales[size_t(n) * ld_scale + 2 * b + 1] = uint8_t(x + 127);
+  *pl.scale_at(n, 2 * b) = uint8_t(x + 127);
+  *pl.scale_at(n, 2 * b + 1) = uint8_t(x + 127);
 }
 
-static cudaError_t launch_pack_mxfp4(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
+static cudaError_t launch_pack_mxfp4(const float* w, int N, int K, const PackPlace& pl, int ld_scale,
                                      float* global_scale, void* ws, cudaStream_t s) {
   unsigned int* amax = static_cast<unsigned int*>(ws);
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), s);
@@ -170,7 +200,7 @@ static cudaError_t launch_pack_mxfp4(const float* w, int N, int K, uint8_t* code
   }
   const long long nthreads = (long long)N * ld_scale;
   ProfileScope prof(FT_KERNEL_PACK, s);
-  mxfp4_pack_kernel<<<dim3(unsigned((nthreads + 255) / 256)), 256, 0, s>>>(w, N, K, codes, scales, ld_scale, amax,
+  mxfp4_pack_kernel<<<dim3(unsigned((nthreads + 255) / 256)), 256, 0, s>>>(w, N, K, pl, ld_scale, amax,
                                                                              global_scale);
   return cudaGetLastError();
 }

@@ -110,6 +110,28 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
+// 4-D tiled TMA load (no multicast).
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, uint64_t* bar, int x, int y, int z,
+                                            int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
+// One weight box (codes: 128 B of each row; scales: 16 B) of 256-K stage ws,
+// rows from y, slot `slot`.  Row-major slots use 3-D maps whose x is the
+// byte column (stage ws starts at ws * stage_bytes); stage-tiled slots use
+// 4-D maps with the stage as a dimension of its own (x = 0).
+__device__ __forceinline__ void tma_load_weights(void* smem_dst, const void* tmap, uint64_t* bar, int tiled,
+                                                 int stage_bytes, int ws, int y, int slot) {
+  if (tiled)
+    tma_load_4d(smem_dst, tmap, bar, 0, y, ws, slot);
+  else
+    tma_load_3d(smem_dst, tmap, bar, ws * stage_bytes, y, slot);
+}
+
 // 2-D tiled TMA load (no multicast).
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, uint64_t* bar, int x, int y) {
   asm volatile(

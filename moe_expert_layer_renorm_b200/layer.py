@@ -9,6 +9,7 @@ from __future__ import annotations
 import ctypes
 from typing import Optional
 
+import numpy as np
 import torch
 
 from . import _lib
@@ -24,13 +25,23 @@ def _stream(s: Optional[torch.cuda.Stream]) -> int:
     return s.cuda_stream
 
 
-class ExpertPool:
-    """A device pool of expert slots (NVFP4, or MXFP4 with fmt=FT_SCALE_MXFP4)
-    laid out by ft_nvfp4_slot_layout_init / ft_mxfp4_slot_layout_init."""
+def untile(block: np.ndarray, N: int, width: int, row_bytes: int) -> np.ndarray:
+    """Stage-tiled bytes [S][N][width] -> row-major [N, row_bytes] (the first
+    row_bytes of each row's S * width bytes)."""
+    S = block.size // (N * width)
+    return np.ascontiguousarray(block.reshape(S, N, width).transpose(1, 0, 2).reshape(N, S * width)[:, :row_bytes])
 
-    def __init__(self, H: int, I: int, num_slots: int, device="cuda", fmt: int = _lib.FT_SCALE_NVFP4):
-        self.H, self.I, self.num_slots, self.fmt = H, I, num_slots, fmt
-        self.layout = _lib.slot_layout(H, I, num_slots, fmt)
+
+class ExpertPool:
+    """A device pool of expert slots (NVFP4, or MXFP4 with fmt=FT_SCALE_MXFP4),
+    row-major or stage-tiled (tiled=True; see ft_tiled_slot_layout_init)."""
+
+    def __init__(self, H: int, I: int, num_slots: int, device="cuda", fmt: int = _lib.FT_SCALE_NVFP4,
+                 tiled: bool = False):
+        self.H, self.I, self.num_slots, self.fmt, self.tiled = H, I, num_slots, fmt, tiled
+        self.layout = _lib.slot_layout(H, I, num_slots, fmt, tiled)
+        # the canonical row-major layout of the same format, for slots read back to the host
+        self.rows_layout = _lib.slot_layout(H, I, num_slots, fmt)
         self.slot_bytes = int(self.layout.slot_bytes)
         self.buf = torch.zeros(num_slots * self.slot_bytes, dtype=torch.uint8, device=device)
         self._pack_ws = torch.zeros(256, dtype=torch.uint8, device=device)
@@ -43,27 +54,44 @@ class ExpertPool:
         return (self.I, self.H) if mat in (FT_GATE, FT_UP) else (self.H, self.I)
 
     def pack_into(self, slot: int, mat: int, w: torch.Tensor, stream=None) -> None:
-        """Quantise fp32 weights w [N, K] (on the device) into `slot`, in the pool's format."""
+        """Quantise fp32 weights w [N, K] (on the device) into `slot`, in the pool's format and layout."""
         N, K = self.shape(mat)
         assert w.shape == (N, K) and w.dtype == torch.float32 and w.is_cuda and w.is_contiguous()
-        L = self.layout
-        base = self.ptr + slot * self.slot_bytes
-        pack = _lib.mxfp4_pack if self.fmt == _lib.FT_SCALE_MXFP4 else _lib.nvfp4_pack
-        pack(w.data_ptr(), N, K, base + L.codes_off[mat], base + L.scales_off[mat], L.ld_scale[mat],
-             base + L.global_off[mat], self._pack_ws.data_ptr(), _stream(stream))
+        _lib.pack_slot(w.data_ptr(), mat, self.layout, self.ptr + slot * self.slot_bytes, self._pack_ws.data_ptr(),
+                       _stream(stream))
 
     def slot_view(self, slot: int) -> torch.Tensor:
         return self.buf[slot * self.slot_bytes:(slot + 1) * self.slot_bytes]
 
     def tensor_bytes(self, slot: int, mat: int):
-        """(codes uint8 [N, K/2], scales uint8 [N, ld], global fp32) of one tensor, on the host."""
+        """(codes uint8 [N, K/2], scales uint8 [N, ld], global fp32) of one tensor, on the host, row-major."""
         N, K = self.shape(mat)
         L = self.layout
+        ld = L.ld_scale[mat]
         s = self.slot_view(slot)
-        codes = s[L.codes_off[mat]:L.codes_off[mat] + N * K // 2].view(N, K // 2).cpu().numpy()
-        scales = s[L.scales_off[mat]:L.scales_off[mat] + N * L.ld_scale[mat]].view(N, L.ld_scale[mat]).cpu().numpy()
+        if self.tiled:
+            S = (K + 255) // 256
+            codes = untile(s[L.codes_off[mat]:L.codes_off[mat] + S * N * 128].cpu().numpy(), N, 128, K // 2)
+            scales = untile(s[L.scales_off[mat]:L.scales_off[mat] + S * N * 16].cpu().numpy(), N, 16, ld)
+        else:
+            codes = s[L.codes_off[mat]:L.codes_off[mat] + N * K // 2].view(N, K // 2).cpu().numpy()
+            scales = s[L.scales_off[mat]:L.scales_off[mat] + N * ld].view(N, ld).cpu().numpy()
         g = s[L.global_off[mat]:L.global_off[mat] + 4].cpu().numpy().view("float32")[0]
         return codes, scales, float(g)
+
+    def export_slot(self, slot: int) -> np.ndarray:
+        """The slot as a host image in the row-major layout `rows_layout`
+        (what the oracle and the host banks read)."""
+        if not self.tiled:
+            return self.slot_view(slot).cpu().numpy()
+        R = self.rows_layout
+        out = np.zeros(int(R.slot_bytes), np.uint8)
+        for mat in range(3):
+            c, sc, g = self.tensor_bytes(slot, mat)
+            out[R.codes_off[mat]:R.codes_off[mat] + c.size] = c.reshape(-1)
+            out[R.scales_off[mat]:R.scales_off[mat] + sc.size] = sc.reshape(-1)
+            out[R.global_off[mat]:R.global_off[mat] + 4] = np.frombuffer(np.float32(g).tobytes(), np.uint8)
+        return out
 
 
 class MoELayer:

@@ -14,10 +14,10 @@ from moe_expert_layer_renorm_b200.layer import ExpertPool, MoELayer
 from oracle import moe_layer as M
 
 
-def build_pool(w: inputs.Workload, layer: int = 0, device="cuda", fmt: int = 0):
+def build_pool(w: inputs.Workload, layer: int = 0, device="cuda", fmt: int = 0, tiled: bool = False):
     s = inputs.layer_seed(w.seed, layer)
     slot_table = inputs.make_slot_table(w.E, w.slots, w.permuted_slots, s)
-    pool = ExpertPool(w.H, w.I, w.slots, device=device, fmt=fmt)
+    pool = ExpertPool(w.H, w.I, w.slots, device=device, fmt=fmt, tiled=tiled)
     for e in range(w.E):
         for mat in range(3):
             N, K = pool.shape(mat)
@@ -95,11 +95,12 @@ def host_pool(pool: ExpertPool, slot_table: np.ndarray, experts):
     """The slots of the given experts copied to the host, packed densely, and
     the slot table that points into that copy (-1 for the other experts)."""
     need = sorted(set(int(v) for v in experts))
-    L = pool.layout
-    buf = np.zeros(max(1, len(need)) * pool.slot_bytes, np.uint8)
+    L = pool.rows_layout           # slots read back in the row-major layout
+    nb = int(L.slot_bytes)
+    buf = np.zeros(max(1, len(need)) * nb, np.uint8)
     table = np.full(len(slot_table), -1, np.int32)
     for i, e in enumerate(need):
-        buf[i * pool.slot_bytes:(i + 1) * pool.slot_bytes] = pool.slot_view(int(slot_table[e])).cpu().numpy()
+        buf[i * nb:(i + 1) * nb] = pool.export_slot(int(slot_table[e]))
         table[e] = i
     return buf, table, L
 
@@ -110,9 +111,9 @@ def reference_y(run: GpuRun, k: int, tok: np.ndarray) -> np.ndarray:
     ids = run.layer.ids.cpu().numpy()
     buf, table, L = host_pool(run.pool, run.slot_table, ids[tok].reshape(-1))
     H, I = run.pool.H, run.pool.I
-    return cpp.moe_layer(run.x_bits, run.logits, k, table, buf, run.pool.slot_bytes, list(L.codes_off),
+    return cpp.moe_layer(run.x_bits, run.logits, k, table, buf, int(L.slot_bytes), list(L.codes_off),
                          list(L.scales_off), list(L.global_off), list(L.ld_scale), H, I, tokens=tok,
-                         fmt=int(run.pool.layout.scale_format))
+                         fmt=int(L.scale_format))
 
 
 def check_output(run: GpuRun, k: int, tokens: Optional[Sequence[int]] = None):

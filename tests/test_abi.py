@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from moe_expert_layer_renorm_b200 import _lib
@@ -135,3 +136,47 @@ def test_mxfp4_layout_is_the_nvfp4_layout_with_its_tag(L):
     for f in ("ld_scale", "codes_off", "scales_off", "global_off"):
         assert list(getattr(a, f)) == list(getattr(b, f))
     assert a.slot_bytes == b.slot_bytes
+
+
+@pytest.mark.parametrize("H,I", [(256, 512), (2048, 768), (2880, 2880), (320, 448)])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_tiled_layout_rules(L, H, I, fmt):
+    lay = _lib.slot_layout(H, I, 3, fmt, tiled=True)
+    rows = (I, I, H)
+    ks = (H, H, I)
+    assert (lay.tiled, lay.scale_format, lay.num_slots) == (1, fmt, 3)
+    ends = []
+    for m in range(3):
+        S = (ks[m] + 255) // 256
+        assert lay.ld_scale[m] == 16 * S
+        assert lay.codes_off[m] % 256 == 0 and lay.scales_off[m] % 256 == 0
+        assert lay.codes_off[m] + S * rows[m] * 128 <= lay.scales_off[m]
+        ends.append(lay.scales_off[m] + S * rows[m] * 16)
+    assert lay.codes_off[1] >= ends[0] and lay.codes_off[2] >= ends[1]
+    assert min(lay.global_off) >= ends[2] and lay.slot_bytes % 256 == 0
+    # when every K is a multiple of 256 the tiled slot has the row-major slot's size
+    if H % 256 == 0 and I % 256 == 0:
+        assert lay.slot_bytes == _lib.slot_layout(H, I, 3, fmt).slot_bytes
+
+
+def test_pack_slot_argument_checks(L):
+    lay = _lib.slot_layout(256, 512, 2, 0, tiled=True)
+    assert L.ft_pack_slot(None, 0, ctypes.byref(lay), None, None, None) == _lib.FT_ERR_INVALID_ARG
+    assert L.ft_pack_slot(None, 3, ctypes.byref(lay), None, None, None) == _lib.FT_ERR_INVALID_ARG
+    bad = _lib.slot_layout(256, 512, 2)
+    bad.tiled = 2
+    assert L.ft_pack_slot(None, 0, ctypes.byref(bad), None, None, None) == _lib.FT_ERR_INVALID_ARG
+    assert L.ft_tiled_slot_layout_init(256, 512, 2, 5, ctypes.byref(bad)) == _lib.FT_ERR_INVALID_ARG
+
+
+def test_untile_reads_stage_tiled_bytes_back_row_major():
+    from moe_expert_layer_renorm_b200.layer import untile
+    g = np.random.default_rng(3)
+    for N, K in ((5, 2880), (3, 512), (1, 64)):
+        S = (K + 255) // 256
+        rows = g.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+        tiled = np.zeros((S, N, 128), np.uint8)
+        for n in range(N):             # by the definition: byte j of row n goes to stage j // 128, column j % 128
+            for j in range(K // 2):
+                tiled[j // 128, n, j % 128] = rows[n, j]
+        assert np.array_equal(untile(tiled.reshape(-1), N, 128, K // 2), rows)

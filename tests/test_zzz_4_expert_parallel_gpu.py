@@ -117,15 +117,15 @@ def _oracle_y(w, pools, G, x_bits, logits, tok):
     pools (the packed bytes the GPU used)."""
     ids, _ = M.route(logits, w.k)
     need = sorted(set(int(e) for e in ids[tok].reshape(-1)))
-    p0 = pools[0]
-    buf = np.zeros(max(1, len(need)) * p0.slot_bytes, np.uint8)
+    L = pools[0].rows_layout        # slots read back row-major
+    nb = int(L.slot_bytes)
+    buf = np.zeros(max(1, len(need)) * nb, np.uint8)
     table = np.full(w.E, -1, np.int32)
     El = w.E // G
     for i, e in enumerate(need):
-        buf[i * p0.slot_bytes:(i + 1) * p0.slot_bytes] = pools[e // El].slot_view(e % El).cpu().numpy()
+        buf[i * nb:(i + 1) * nb] = pools[e // El].export_slot(e % El)
         table[e] = i
-    L = p0.layout
-    return cpp.moe_layer(x_bits, logits, w.k, table, buf, p0.slot_bytes, list(L.codes_off), list(L.scales_off),
+    return cpp.moe_layer(x_bits, logits, w.k, table, buf, nb, list(L.codes_off), list(L.scales_off),
                          list(L.global_off), list(L.ld_scale), w.H, w.I, tokens=tok)
 
 
