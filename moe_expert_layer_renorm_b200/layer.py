@@ -57,8 +57,14 @@ class ExpertPool:
         """Quantise fp32 weights w [N, K] (on the device) into `slot`, in the pool's format and layout."""
         N, K = self.shape(mat)
         assert w.shape == (N, K) and w.dtype == torch.float32 and w.is_cuda and w.is_contiguous()
-        _lib.pack_slot(w.data_ptr(), mat, self.layout, self.ptr + slot * self.slot_bytes, self._pack_ws.data_ptr(),
-                       _stream(stream))
+        base = self.ptr + slot * self.slot_bytes
+        if self.tiled:
+            _lib.pack_slot(w.data_ptr(), mat, self.layout, base, self._pack_ws.data_ptr(), _stream(stream))
+            return
+        L = self.layout
+        pack = _lib.mxfp4_pack if self.fmt == _lib.FT_SCALE_MXFP4 else _lib.nvfp4_pack
+        pack(w.data_ptr(), N, K, base + L.codes_off[mat], base + L.scales_off[mat], L.ld_scale[mat],
+             base + L.global_off[mat], self._pack_ws.data_ptr(), _stream(stream))
 
     def slot_view(self, slot: int) -> torch.Tensor:
         return self.buf[slot * self.slot_bytes:(slot + 1) * self.slot_bytes]

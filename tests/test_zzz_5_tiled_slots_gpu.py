@@ -2,7 +2,9 @@
 row-major slots, arranged so that each weight box the GEMMs load is one
 contiguous block.  The packed tensors read back identical to row-major
 packing, and the layer gives bit-identical outputs on both layouts (the
-kernels only load from other addresses), and matches the oracle."""
+kernels only load from other addresses), and matches the oracle.
+
+Collected last: the layout is new and has not yet run on a B200."""
 import numpy as np
 import pytest
 import torch
@@ -72,3 +74,18 @@ def test_mxfp4_layer_on_tiled_slots(cuda_device):
     a = G.run_gpu(w, pool=pool_r, slot_table=st, li=li)
     b = G.run_gpu(w, pool=pool_t, slot_table=st, li=li)
     assert np.array_equal(a.y, b.y)
+
+
+def test_pack_slot_row_major_equals_the_plain_pack(cuda_device):
+    # ft_pack_slot on a row-major layout places the bytes as ft_nvfp4_pack does
+    H, I = 2880, 2880
+    a = ExpertPool(H, I, 1)
+    b = ExpertPool(H, I, 1)
+    for mat in range(3):
+        N, K = a.shape(mat)
+        wt = inputs.make_weight_fp32_torch(N, K, 78, 2, mat, "cuda")
+        a.pack_into(0, mat, wt)
+        _lib.pack_slot(wt.data_ptr(), mat, b.layout, b.ptr, b._pack_ws.data_ptr(),
+                       torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert torch.equal(a.buf, b.buf)
