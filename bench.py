@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"], help="expert weight format")
     ap.add_argument("--layout", default="rows", choices=["rows", "tiled"],
                     help="expert slot layout: row-major tensors, or stage-tiled (each weight box contiguous)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: the experts split over the ranks, rows exchanged all-to-all "
+                         "(each rank still brings its own tokens: weak scaling)")
     ap.add_argument("--fused-front", action="store_true",
                     help="route and permute through ft_moe_route_permute (one launch for small batches)")
     ap.add_argument("--slot-churn", nargs="?", const="decode", default=None, choices=["decode", "prefill_stream"],
@@ -721,12 +724,83 @@ def run_prefill_stream():
         "stats": r["stats"]}))
 
 
+def run_ep(args):
+    """The layer with its experts split over the ranks (ExpertParallelMoE over
+    NCCL; a one-rank group when run without torchrun).  Every rank routes its
+    own batch; the step is eager (the exchange plan needs the routed counts on
+    the host), timed with CUDA events, max over ranks."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    from moe_expert_layer_renorm_b200.ep import ExpertParallelMoE, owned_experts
+    from moe_expert_layer_renorm_b200.layer import ExpertPool
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    else:
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = inputs.WORKLOADS[args.workload]
+    mine = owned_experts(w.E, world, rank)
+    from moe_expert_layer_renorm_b200 import _lib
+    pool = ExpertPool(w.H, w.I, len(mine), device=dev, tiled=args.layout == "tiled",
+                      fmt=_lib.FT_SCALE_MXFP4 if args.fmt == "mxfp4" else _lib.FT_SCALE_NVFP4)
+    for j, e in enumerate(mine):                     # the same experts as one GPU would hold, split by owner
+        for mat in range(3):
+            N, K = pool.shape(mat)
+            pool.pack_into(j, mat, inputs.make_weight_fp32_torch(N, K, w.seed, e, mat, dev))
+    table = torch.arange(len(mine), dtype=torch.int32, device=dev)
+    li = inputs.make_layer_inputs(inputs.custom_workload(w, seed=rank_layer_seed(w, rank, 0)), 0)
+    x = torch.from_numpy(li.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    lg = torch.from_numpy(li.logits).to(dev)
+    ep = ExpertParallelMoE(w.T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev)
+    for _ in range(max(3, args.warmup)):
+        ep.forward(x, lg, table, pool)
+    dist.barrier()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    recv = 0
+    for _ in range(args.steps):
+        ep.forward(x, lg, table, pool)
+        recv += ep.plan.n_recv
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), dev)
+    line = {"metric": "MoE-layer tokens/s, experts split over the ranks", "value": round(world * w.T * args.steps /
+                                                                                        (ms * 1e-3), 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": f"{args.fmt} weights, f16 MMA operands, fp32 accumulate",
+            "data": "synthetic (seeded; each rank its own batch, the experts of one layer split by owner)",
+            "config": dict(run_config(args, {"workload": w.name, "T_per_rank": w.T, "E": w.E, "k": w.k, "H": w.H,
+                                             "I": w.I}),
+                           parallelism=f"ep{world}", experts_per_rank=len(mine),
+                           rows_received_per_step_rank0=round(recv / args.steps, 1),
+                           timing="eager steps (one host synchronisation per step for the exchange plan)")}
+    dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
     elif args.slot_churn:
         run_slot_churn(args)
+    elif args.ep:
+        run_ep(args)
     else:
         run_ours(args)
 
