@@ -113,6 +113,8 @@ class ExpertParallelMoE:
         self.x_send = torch.empty((T * k, H), dtype=torch.bfloat16, device=self.device)
         self.ffn_ws = torch.empty(256, dtype=torch.uint8, device=self.device)
         self.plan: Optional[ExchangePlan] = None
+        self._pin: Optional[torch.Tensor] = None    # page-locked staging of the plan's index arrays
+        self._idx: Optional[torch.Tensor] = None
 
     def _workspace(self, n_recv: int) -> torch.Tensor:
         need = _lib.ffn_workspace_size(n_recv, self.H, self.I, self.E_local, 1)
@@ -139,9 +141,19 @@ class ExpertParallelMoE:
         plan = self.plan = ExchangePlan(self.exchange.gather_offsets(L.offsets), self.G, self.E, self.rank)
         n = plan.n_recv
         dev = self.device
-        perm_src_local = torch.from_numpy(plan.perm_src_local).to(dev, non_blocking=False)
-        ret_idx = torch.from_numpy(plan.ret_idx).to(dev, non_blocking=False)
-        local_offsets = torch.from_numpy(plan.local_offsets).to(dev, non_blocking=False)
+        # the plan's three index arrays: one page-locked buffer, one copy (the next step's offsets
+        # exchange waits on the stream before this buffer is written again)
+        m, El = max(n, 1), self.E_local
+        need = 2 * m + El + 1
+        if self._pin is None or self._pin.numel() < need:
+            self._pin = torch.empty(need, dtype=torch.int32, pin_memory=True)
+            self._idx = torch.empty(need, dtype=torch.int32, device=dev)
+        hp = self._pin.numpy()
+        hp[:m] = plan.perm_src_local
+        hp[m:2 * m] = plan.ret_idx
+        hp[2 * m:need] = plan.local_offsets
+        self._idx[:need].copy_(self._pin[:need], non_blocking=True)
+        perm_src_local, ret_idx, local_offsets = self._idx[:m], self._idx[m:2 * m], self._idx[2 * m:need]
 
         x_recv = torch.empty((max(n, 1), H), dtype=torch.bfloat16, device=dev)
         self.exchange.rows(x_recv[:n], self.x_send, plan.recv_rows, plan.send_rows)
