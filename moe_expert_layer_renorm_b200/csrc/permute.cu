@@ -45,7 +45,11 @@ __device__ int block_exclusive_scan(int v, int* smem_warp_sums) {
 }
 
 // Walk pairs [p0, p1) in order with one warp; cursor[e] is this chunk's next
-// row for expert e (shared memory), advanced as pairs are placed.
+// row for expert e (shared memory), advanced as pairs are placed.  With
+// SMEM_IDS the ids are read from a shared-memory copy indexed from p0 (the
+// single-CTA path loads them once, in parallel, instead of one dependent
+// global round trip per 32 pairs).
+template <bool SMEM_IDS>
 __device__ void scatter_chunk_warp(const int32_t* __restrict__ ids, int p0, int p1, int E, int* cursor,
                                    int32_t* __restrict__ perm_src, int32_t* __restrict__ pair_to_row,
                                    int P) {
@@ -53,7 +57,7 @@ __device__ void scatter_chunk_warp(const int32_t* __restrict__ ids, int p0, int 
   for (int base = p0; base < p1; base += 32) {
     const int p = base + lane;
     const bool live = p < p1;
-    int e = live ? __ldg(ids + p) : -1;
+    int e = live ? (SMEM_IDS ? ids[p - p0] : __ldg(ids + p)) : -1;
     if (live && !valid_expert(e, E)) { set_device_status(FT_DEV_BAD_INDEX); e = -1; }
     const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
@@ -78,10 +82,12 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
   pdl_enter();
   __shared__ int cnt[kMaxExperts];
   __shared__ int warp_sums[32];
+  __shared__ int32_t sids[kPermChunk];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int p = threadIdx.x; p < P; p += blockDim.x) {
     const int e = __ldg(ids + p);
+    sids[p] = e;
     if (valid_expert(e, E)) atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
@@ -92,7 +98,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
   if (e < E) { offsets[e] = ex; cnt[e] = ex; }
   if (e == E - 1) offsets[E] = ex + c;
   __syncthreads();
-  if (threadIdx.x < 32) scatter_chunk_warp(ids, 0, P, E, cnt, perm_src, pair_to_row, P);
+  if (threadIdx.x < 32) scatter_chunk_warp<true>(sids, 0, P, E, cnt, perm_src, pair_to_row, P);
 }
 
 __global__ void __launch_bounds__(256) permute_hist_kernel(const int32_t* __restrict__ ids, int P, int E,
@@ -143,7 +149,7 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __r
   __syncthreads();
   if (threadIdx.x < 32) {
     const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
-    scatter_chunk_warp(ids, p0, p1, E, cursor, perm_src, pair_to_row, P);
+    scatter_chunk_warp<false>(ids, p0, p1, E, cursor, perm_src, pair_to_row, P);
   }
 }
 
