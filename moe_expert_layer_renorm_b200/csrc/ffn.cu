@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0,
                 const __grid_constant__ CUtensorMap tm_scales0, const __grid_constant__ CUtensorMap tm_codes1,
                 const __grid_constant__ CUtensorMap tm_scales1, const __grid_constant__ CUtensorMap tm_act) {
-  pdl_enter();
+  pdl_wait();   // dependents are triggered at the end (see below)
   using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB, KC>;
   constexpr int kCPW = Cfg::kCPW;
   extern __shared__ uint8_t smem_raw[];
@@ -580,6 +580,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
 
   tc_fence_before();
   __syncthreads();
+  pdl_launch_dependents();   // the next kernel's CTAs may now take this SM's place
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -280,6 +280,13 @@ __device__ __forceinline__ void pdl_enter() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// The two halves separately: a kernel that fills whole SMs triggers its
+// dependents only as its CTAs finish, so that their early CTAs do not take
+// SM resources from it while it runs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // Launch with the programmatic-stream-serialisation attribute: the kernel
 // may start before the previous kernel in the stream ends, and waits for it
