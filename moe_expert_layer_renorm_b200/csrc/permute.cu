@@ -162,28 +162,6 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __r
 constexpr int kFusedMaxT = 128;
 constexpr int kFusedMaxE = 512;
 
-// One warp places pairs 0 .. P-1 in order; ids in shared memory, cursor[e] the
-// next row of expert e.
-__device__ void scatter_smem_warp(const int* s_ids, int P, int* cursor, int32_t* __restrict__ perm_src,
-                                  int32_t* __restrict__ pair_to_row) {
-  const int lane = threadIdx.x & 31;
-  for (int base = 0; base < P; base += 32) {
-    const int p = base + lane;
-    const int e = p < P ? s_ids[p] : -1;
-    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    const int leader = __ffs(peers) - 1;
-    const int row = e >= 0 ? cursor[e] + rank : -1;
-    __syncwarp();
-    if (e >= 0 && lane == leader) cursor[e] += __popc(peers);
-    __syncwarp();
-    if (row >= 0 && row < P) {
-      perm_src[row] = p;
-      pair_to_row[p] = row;
-    }
-  }
-}
-
 template <int NPL>
 __global__ void __launch_bounds__(1024) route_permute_small_kernel(const float* __restrict__ logits, int T, int E,
                                                                    int k, int mode, int32_t* __restrict__ ids,
@@ -217,7 +195,7 @@ __global__ void __launch_bounds__(1024) route_permute_small_kernel(const float* 
   if (e < E) { offsets[e] = ex; cnt[e] = ex; }
   if (e == E - 1) offsets[E] = ex + c;
   __syncthreads();
-  if (warp == 0) scatter_smem_warp(s_ids, P, cnt, perm_src, pair_to_row);
+  if (warp == 0) scatter_chunk_warp<true>(s_ids, 0, P, E, cnt, perm_src, pair_to_row, P);
 }
 
 static bool route_permute_fused_fits(int T, int k, int E) {
