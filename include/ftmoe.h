@@ -199,10 +199,12 @@ FT_API int ft_moe_route_permute(const float* logits, int T, int E, int k, int mo
  * ceil(T*k / 1024) * E <= 65536 (always met when T*k <= 1024); larger inputs
  * return FT_ERR_INVALID_ARG and launch nothing.  The array needs no zeroing.
  *
- * The first call with a given device current looks up that device's copy of
- * the array; make it before any stream capture.  Calls on one device share
- * the array: two calls that can overlap in time (different streams, or
- * different host threads) race and give wrong rows, so order them.
+ * Every call looks up the current device's copy of the array (a host-side
+ * query, valid across devices and after a device reset); the first call on
+ * a device may load the library's device code there, so make it before any
+ * stream capture.  Calls on one device share the array: two calls that can
+ * overlap in time (different streams, or different host threads) race and
+ * give wrong rows, so order them.
  * Arguments are those of ft_moe_permute minus ws and ws_bytes.
  */
 FT_API int ft_moe_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
@@ -217,12 +219,19 @@ FT_API int ft_moe_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
  *   out_perm[r] = gD * (Qd h[r])                                (H values, fp32)
  * where Q* are the E2M1*E4M3 dequantised weights, g* the fp32 global scales,
  * and products accumulate in fp32 on the tensor cores.  The MMA operands are
- * f16: every E2M1*E4M3 product is exact in f16; each token row of x is
- * converted once, after a power-of-two prescale that puts its largest
- * magnitude below 2^15 (exact for every element within 2^32 of that
- * maximum, else an absolute error below 2^-41 of it); h is rounded to f16
- * (values beyond the f16 range saturate and set FT_DEV_F16_RANGE).  The
- * expert outputs stay fp32 so that the layer output meets
+ * f16:
+ *   - every E2M1*E4M3 product is exact in f16;
+ *   - each token row x_t is converted once, times the power of two 2^(12-e)
+ *     that puts its largest magnitude in [2^14, 2^15) (e: max|x_t| * 2^-e in
+ *     [4, 8); any finite bf16 row has one).  Elements within a factor 2^31 of
+ *     the row's largest magnitude convert exactly; smaller ones round with an
+ *     absolute error of at most 2^-39 max|x_t|;
+ *   - h is rounded to f16 after dividing it by 2^(2e), the square of its
+ *     row's factor (undone exactly, in fp32, on the down projection's
+ *     output), so its range does not depend on the row's magnitude, only
+ *     on the weights and the row's shape.  A normalised h beyond +-65504
+ *     saturates and sets FT_DEV_F16_RANGE.
+ * The expert outputs stay fp32 so that the layer output meets
  * |y - y_exact| <= 1e-2 rms(y) + 1e-3: a bf16 rounding of them (or of y) alone
  * would already reach that bound at the tails of the output distribution.
  *   x              device bf16 [T, H]

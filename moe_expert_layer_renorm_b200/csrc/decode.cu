@@ -243,7 +243,7 @@ __device__ __forceinline__ bool dec_epilogue(const DecodeParams& p, const DecUni
         const int r = 8 * n + 2 * t + e;
         if (r < d.nr && f < G.M) {
           store_out<2>(G.out, size_t(d.rb + r) * G.M + f,
-                       silu_mul(c.g0 * ts[n][e] * acc[n][e], c.g1 * ts[n][e] * acc[n][2 + e]));
+                       silu_mul(c.g0 * kRowNormInv * acc[n][e], c.g1 * kRowNormInv * acc[n][2 + e], ts[n][e]));
         }
       }
   } else {
@@ -255,8 +255,8 @@ __device__ __forceinline__ bool dec_epilogue(const DecodeParams& p, const DecUni
         const int r = 8 * n + 2 * t + e;
         if (r < d.nr) {
           float* o = static_cast<float*>(G.out) + size_t(d.rb + r) * G.M;
-          if (f < G.M) o[f] = c.g0 * acc[n][e];
-          if (f + 8 < G.M) o[f + 8] = c.g0 * acc[n][2 + e];
+          if (f < G.M) o[f] = down_out(c.g0, acc[n][e], ts[n][e]);
+          if (f + 8 < G.M) o[f + 8] = down_out(c.g0, acc[n][2 + e], ts[n][e]);
         }
       }
   }
@@ -286,14 +286,15 @@ __device__ bool dec_unit(const DecodeParams& p, const DecUnit& d, uint8_t* smem,
     blo = mx_bias(__ldg(reinterpret_cast<const float*>(sbase + G.global_off[0])));
     bhi = mx_bias(__ldg(reinterpret_cast<const float*>(sbase + G.global_off[1])));
   }
-  // gate/up: the factors undoing the token rows' prescale, loaded now, used in the epilogue
+  // the token rows' factors f_r (see silu_mul), loaded now, used in the epilogue
   float ts[NT][2];
+  const float* rs = p.g[d.gemm].rowscale;
 #pragma unroll
   for (int n = 0; n < NT; ++n)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int r = 8 * n + 2 * t + e;
-      ts[n][e] = d.gemm == 0 && r < d.nr ? __ldg(p.g[0].rowscale + d.rb + r) : 1.0f;
+      ts[n][e] = rs != nullptr && r < d.nr ? __ldg(rs + d.rb + r) : 1.0f;
     }
   float acc[NT][4];
 #pragma unroll

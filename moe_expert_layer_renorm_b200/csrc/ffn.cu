@@ -45,7 +45,7 @@ constexpr int kMatStageBytes = kCodesBytes + kScaleBytes;   // 18 KB, multiple o
 constexpr int kThreads = 512;
 
 struct FfnParams {
-  const float* rowscale;      // GEMM1: per permuted row, the factor undoing the f16 prescale of x; GEMM2: null
+  const float* rowscale;      // per permuted row, its factor f_r = 2^e_r (see silu_mul); null reads as 1
   const int32_t* perm_src;    // GEMM1: row -> pair (token = pair / k_top); GEMM2: null (row -> row)
   int k_top;
   int K;                      // reduction length
@@ -189,10 +189,28 @@ struct Abort {
   }
 };
 
-// silu(g) * u = g * u / (1 + e^-g).  The hardware exponential and a fast
-// divide: a few ulps of fp32, far inside the layer's tolerance; as g -> -inf
-// the divisor overflows to inf and the result goes to 0, its limit.
-__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g * u, 1.0f + __expf(-g)); }
+// Per-row normalisation of the token rows.  Row r (token t) has the
+// exponent e_r with max|x_t| * 2^-e_r in [4, 8) (e_r = 0 for an all-zero row),
+// and rowscale[r] = f_r = 2^e_r.  GEMM1 multiplies f16 operands
+// x' = x * 2^(12 - e_r) (largest magnitude in [2^14, 2^15)), so with the
+// global scale gG its accumulator gives G' = gG * 2^-12 * acc = G / f_r: the
+// gate (and likewise the up) projection of the row scaled to a largest
+// magnitude in [4, 8).  h is stored normalised the same way,
+//   h' = silu(G) * U / f_r^2 = G' * U' / (1 + e^-(G' f_r)),
+// so its f16 range does not depend on the row's magnitude, and GEMM2 undoes
+// it exactly: out = (gD * acc * f_r) * f_r.  For rows of largest magnitude in
+// [4, 8) (the N(0, 1) workloads) f_r = 1 and nothing changes.
+constexpr float kRowNormInv = 1.0f / 4096.0f;   // 2^-12
+
+// h' = g * u / (1 + e^-(g f)).  The hardware exponential and a fast divide: a
+// few ulps of fp32, far inside the layer's tolerance; as g f -> -inf the
+// divisor overflows to inf and the result goes to 0, its limit.
+__device__ __forceinline__ float silu_mul(float g, float u, float f) {
+  return __fdividef(g * u, 1.0f + __expf(-(g * f)));
+}
+// GEMM2's output from its accumulator: (gD * acc * f) * f, in this order so
+// that no intermediate leaves the fp32 range when the result does not.
+__device__ __forceinline__ float down_out(float gd, float acc, float f) { return (gd * acc * f) * f; }
 
 // GEMM1 stores h in f16 (it is the next MMA's operand; a value beyond the f16
 // range saturates and records FT_DEV_F16_RANGE); GEMM2 stores the expert
@@ -210,8 +228,7 @@ __device__ __forceinline__ void store_out(void* out, size_t idx, float v) {
   }
 }
 
-// Factor undoing the power-of-two prescale of permuted row `row` (GEMM1; 1
-// for GEMM2, whose input h carries no prescale).
+// The row factor f_r of permuted row `row` (1 without a rowscale array).
 __device__ __forceinline__ float token_factor(const FfnParams& p, int row) {
   return p.rowscale != nullptr ? __ldg(p.rowscale + row) : 1.0f;
 }
@@ -479,15 +496,19 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
       float gsc[NMAT];
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) gsc[m] = __ldg(reinterpret_cast<const float*>(sbase + p.global_off[m]));
+      if (NMAT == 2) {   // G' and U' of the normalised rows (exact: a power of two)
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) gsc[m] *= kRowNormInv;
+      }
       const bool split = p.splits > 1;
-      // prescale factors of the unit's token rows, one coalesced load per 32
-      // rows issued before the accumulators are ready; lane j of group g holds
+      // row factors of the unit's token rows, one coalesced load per 32 rows
+      // issued before the accumulators are ready; lane j of group g holds
       // row 32 g + j and the block loop broadcasts them with shuffles
       constexpr int kGroups = (BN + 31) / 32;
       float tsl[kGroups];
 #pragma unroll
       for (int g = 0; g < kGroups; ++g)
-        tsl[g] = NMAT == 2 && !split && g * 32 + lane < nr ? token_factor(p, rb + g * 32 + lane) : 1.0f;
+        tsl[g] = !split && g * 32 + lane < nr ? token_factor(p, rb + g * 32 + lane) : 1.0f;
       if (!(ok = __all_sync(0xFFFFFFFFu, ab.wait(&d_full[ds], (di / DB) & 1, kTagDFull, di, u)))) break;
       tc_fence_after();
       const int n_eff = (nr + 15) & ~15;
@@ -528,9 +549,9 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
           } else if (feat < p.M) {
             float r;
             if (NMAT == 2) {
-              r = silu_mul(gsc[0] * ts * __uint_as_float(w[0][i]), gsc[NMAT - 1] * ts * __uint_as_float(w[NMAT - 1][i]));
+              r = silu_mul(gsc[0] * __uint_as_float(w[0][i]), gsc[NMAT - 1] * __uint_as_float(w[NMAT - 1][i]), ts);
             } else {
-              r = gsc[0] * __uint_as_float(w[0][i]);
+              r = down_out(gsc[0], __uint_as_float(w[0][i]), ts);
             }
             store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
           }
@@ -563,11 +584,11 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
             }
             if (feat < p.M) {
               float r;
+              const float ts = token_factor(p, rb + n);
               if (NMAT == 2) {
-                const float ts = token_factor(p, rb + n);
-                r = silu_mul(gsc[0] * ts * acc[0], gsc[NMAT - 1] * ts * acc[NMAT - 1]);
+                r = silu_mul(gsc[0] * acc[0], gsc[NMAT - 1] * acc[NMAT - 1], ts);
               } else {
-                r = gsc[0] * acc[0];
+                r = down_out(gsc[0], acc[0], ts);
               }
               store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
             }
@@ -694,38 +715,45 @@ __device__ void prep_schedule(const PrepParams& p, int b) {
 __device__ __forceinline__ float bf16x2_absmax(uint32_t w) {
   return fmaxf(fabsf(__uint_as_float(w << 16)), fabsf(__uint_as_float(w & 0xFFFF0000u)));
 }
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& v, float f) {
+// x * fa * fb to f16, eight values.  fa, fb are powers of two (two factors, so
+// that a scaling by up to 2^147 needs no factor outside the fp32 range).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& v, float fa, float fb) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const __half2 h = __floats2half2_rn(__uint_as_float(w[q] << 16) * f, __uint_as_float(w[q] & 0xFFFF0000u) * f);
+    const __half2 h = __floats2half2_rn(__uint_as_float(w[q] << 16) * fa * fb,
+                                        __uint_as_float(w[q] & 0xFFFF0000u) * fa * fb);
     o[q] = *reinterpret_cast<const uint32_t*>(&h);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// The row's prescale shift from its largest magnitude (warp-wide max first).
-__device__ __forceinline__ int prep_shift(float m) {
+// The row exponent e_r from the row's largest magnitude m (warp-wide max
+// first): m * 2^-e_r in [4, 8); 0 for an all-zero row, and for a non-finite
+// one, which also records FT_DEV_F16_RANGE.
+__device__ __forceinline__ int prep_row_exp(float m) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-  int shift = 0;
-  if (m >= 32768.0f && m <= 3.0e38f) {          // finite and too large for f16
-    int e;
-    frexpf(m, &e);                               // m = f * 2^e, f in [0.5, 1)
-    shift = e - 15;                              // m * 2^-shift < 2^15
-  } else if (!(m <= 3.0e38f)) {
+  if (!(m <= 3.4028235e38f)) {
     set_device_status(FT_DEV_F16_RANGE);         // inf or nan input
+    return 0;
   }
-  return shift;
+  if (m == 0.0f) return 0;
+  int e;
+  frexpf(m, &e);                                 // m = f * 2^e, f in [0.5, 1); exact for subnormals too
+  return e - 3;                                  // m * 2^-(e - 3) = 8 f in [4, 8)
 }
 
 // One warp per permuted row r (token t = perm_src[r] / k): writes
-// x_perm[r] = f16(x[t] * 2^-s_t) and rowscale[r] = 2^s_t, with s_t >= 0 the
-// smallest shift that brings max|x[t]| below 2^15.  The f16 conversion is
-// then exact for every element of the row within a factor 2^32 of the row's
-// largest magnitude (bf16 has 8 significant bits, f16 subnormals reach
-// 2^-24); smaller elements round with an absolute error below 2^-41 max|x[t]|.
+// x_perm[r] = f16(x[t] * 2^(12 - e_r)) and rowscale[r] = 2^e_r, e_r the row
+// exponent (max|x[t]| * 2^-e_r in [4, 8), so the converted row's largest
+// magnitude is in [2^14, 2^15)).  Every finite bf16 row qualifies (e_r in
+// [-135, 125]).  The f16 conversion is exact for every element of the row
+// within a factor 2^31 of the row's largest magnitude (bf16 has 8
+// significant bits; f16 represents those exactly down to 2^-17); smaller
+// elements round, to f16 subnormals, with an absolute error of at most
+// 2^-25 in converted units, below 2^-39 max|x[t]|.
 // Rows in permuted order make each expert group's tokens one contiguous
 // block, so the GEMM loads them as plain tiles.  Rows of up to 3072 values
 // are read once into registers with all loads in flight together (the
@@ -751,13 +779,14 @@ __device__ void prep_rows(const PrepParams& p, int b) {
     for (int i = 0; i < kRegVec; ++i)
       m = fmaxf(m, fmaxf(fmaxf(bf16x2_absmax(v[i].x), bf16x2_absmax(v[i].y)),
                          fmaxf(bf16x2_absmax(v[i].z), bf16x2_absmax(v[i].w))));
-    const int shift = prep_shift(m);
-    const float f = ldexpf(1.0f, -shift);
-    if (lane == 0) p.rowscale[r] = ldexpf(1.0f, shift);
+    const int e = prep_row_exp(m);
+    const int sx = 12 - e, sa = sx >> 1;
+    const float fa = ldexpf(1.0f, sa), fb = ldexpf(1.0f, sx - sa);
+    if (lane == 0) p.rowscale[r] = ldexpf(1.0f, e);
 #pragma unroll
     for (int i = 0; i < kRegVec; ++i) {
       const int c = lane + 32 * i;
-      if (c < nv) out[c] = bf16x8_to_f16x8(v[i], f);
+      if (c < nv) out[c] = bf16x8_to_f16x8(v[i], fa, fb);
     }
     return;
   }
@@ -766,10 +795,11 @@ __device__ void prep_rows(const PrepParams& p, int b) {
     const uint4 v = __ldg(row + c);
     m = fmaxf(m, fmaxf(fmaxf(bf16x2_absmax(v.x), bf16x2_absmax(v.y)), fmaxf(bf16x2_absmax(v.z), bf16x2_absmax(v.w))));
   }
-  const int shift = prep_shift(m);
-  const float f = ldexpf(1.0f, -shift);
-  if (lane == 0) p.rowscale[r] = ldexpf(1.0f, shift);
-  for (int c = lane; c < nv; c += 32) out[c] = bf16x8_to_f16x8(__ldg(row + c), f);
+  const int e = prep_row_exp(m);
+  const int sx = 12 - e, sa = sx >> 1;
+  const float fa = ldexpf(1.0f, sa), fb = ldexpf(1.0f, sx - sa);
+  if (lane == 0) p.rowscale[r] = ldexpf(1.0f, e);
+  for (int c = lane; c < nv; c += 32) out[c] = bf16x8_to_f16x8(__ldg(row + c), fa, fb);
 }
 
 __global__ void __launch_bounds__(256, 2) ffn_prep_kernel(const PrepParams p) {

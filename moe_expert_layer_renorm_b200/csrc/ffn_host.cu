@@ -319,7 +319,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
 
   FfnParams p2 = p1;
   p2.perm_src = nullptr;
-  p2.rowscale = nullptr;
+  p2.rowscale = rowscale;   // the same permuted rows: GEMM2 undoes the rows' normalisation of h
   p2.K = I;
   p2.M = H;
   p2.nkw = pl.nkw2;

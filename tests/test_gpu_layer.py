@@ -71,11 +71,15 @@ def test_wide_experts_sampled(cuda_device):
 
 
 def test_wide_decode_sweep_layers(cuda_device):
+    # every layer of the 48-layer sweep (independent seeded weights and inputs), each checked on its own
     w = W["wide_decode_T1"]
-    for layer in (0, 1, 47):
+    assert inputs.WIDE_SWEEP_LAYERS == 48
+    for layer in range(inputs.WIDE_SWEEP_LAYERS):
         run = G.run_gpu(w, layer=layer)
         G.check_routing(run, w.k)
         G.check_output(run, w.k)
+        del run
+        torch.cuda.empty_cache()
 
 
 def test_all_tokens_one_expert(cuda_device):
