@@ -14,38 +14,26 @@
 // kernels of the same call read, so the scratch needs no zeroing, at start-up
 // or between calls.
 //
-// The device address of the scratch is looked up once per device, on the
-// first call made with that device current; make that first call before any
-// stream capture.  All calls on one device share the one scratch array, so
-// two calls that may run at the same time (on two streams, or from two host
-// threads) race on it: order them on one stream or with events.
-#include <atomic>
-
+// The device address of the scratch is looked up on every call that needs
+// it, with the caller's device current (a host-side lookup, cheap next to the
+// launches), so it stays right across devices and after a device reset.  The
+// first call on a device may load this module's device code there: make it
+// before any stream capture.  All calls on one device share the one scratch
+// array, so two calls that may run at the same time (on two streams, or from
+// two host threads) race on it: order them on one stream or with events.
 #include "ftmoe.h"
 
 namespace ftmoe {
 
 constexpr int kNoAllocScratchInts = 65536;
-constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocScratchInts];
 
-static std::atomic<int32_t*> g_permute_scratch_addr[kNoAllocMaxDevices];
-
-// Device address of g_permute_scratch on the current device (set-up on first use).
+// Device address of g_permute_scratch on the current device.  In host code
+// the array's name stands for the host-side shadow of the symbol, not a
+// device address, so it is never passed to a kernel directly.
 static cudaError_t permute_scratch(int32_t** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
-  int32_t* p = g_permute_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_permute_scratch);
-    if (e != cudaSuccess) return e;
-    g_permute_scratch_addr[dev].store(p, std::memory_order_release);
-  }
-  *out = p;
-  return cudaSuccess;
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_permute_scratch);
 }
 
 }  // namespace ftmoe
@@ -68,17 +56,12 @@ extern "C" int ft_moe_permute_noalloc(const int32_t* ids, int T, int k, int E, i
     const cudaError_t e = cudaMemsetAsync(offsets, 0, size_t(E + 1) * sizeof(int32_t), s);
     return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_permute_noalloc");
   }
-  if (nchunks <= 1) {
-    permute_small_kernel<<<1, 1024, 0, s>>>(ids, int(P), E, offsets, perm_src, pair_to_row);
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_permute_noalloc");
-  }
   int32_t* counts = nullptr;
-  cudaError_t e = permute_scratch(&counts);
-  if (e != cudaSuccess) return cuda_fail(e, "ft_moe_permute_noalloc: scratch set-up");
-  permute_hist_kernel<<<int(nchunks), 256, 0, s>>>(ids, int(P), E, counts);
-  permute_scan_kernel<<<1, 1024, 0, s>>>(counts, int(nchunks), E, offsets);
-  permute_scatter_kernel<<<int(nchunks), 256, 0, s>>>(ids, int(P), E, counts, perm_src, pair_to_row);
-  e = cudaGetLastError();
+  if (nchunks > 1) {
+    const cudaError_t e = permute_scratch(&counts);
+    if (e != cudaSuccess) return cuda_fail(e, "ft_moe_permute_noalloc: scratch address");
+  }
+  // the launches of ft_moe_permute, with the scratch in place of the workspace
+  const cudaError_t e = launch_permute(ids, T, k, E, offsets, perm_src, pair_to_row, counts, s);
   return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_permute_noalloc");
 }

@@ -115,6 +115,11 @@ class ExpertParallelMoE:
         self.plan: Optional[ExchangePlan] = None
         self._pin: Optional[torch.Tensor] = None    # page-locked staging of the plan's index arrays
         self._idx: Optional[torch.Tensor] = None
+        # ordering of the two staging buffers across calls, whatever streams the calls use:
+        # the host rewrites _pin only after the previous copy out of it has run, and the copy
+        # into _idx waits until the previous step's kernels have stopped reading _idx
+        self._pin_copied: Optional[torch.cuda.Event] = None
+        self._idx_free: Optional[torch.cuda.Event] = None
 
     def _workspace(self, n_recv: int) -> torch.Tensor:
         need = _lib.ffn_workspace_size(n_recv, self.H, self.I, self.E_local, 1)
@@ -141,18 +146,24 @@ class ExpertParallelMoE:
         plan = self.plan = ExchangePlan(self.exchange.gather_offsets(L.offsets), self.G, self.E, self.rank)
         n = plan.n_recv
         dev = self.device
-        # the plan's three index arrays: one page-locked buffer, one copy (the next step's offsets
-        # exchange waits on the stream before this buffer is written again)
+        # the plan's three index arrays: one page-locked buffer, one copy
         m, El = max(n, 1), self.E_local
         need = 2 * m + El + 1
+        if self._pin_copied is not None:
+            self._pin_copied.synchronize()
         if self._pin is None or self._pin.numel() < need:
             self._pin = torch.empty(need, dtype=torch.int32, pin_memory=True)
             self._idx = torch.empty(need, dtype=torch.int32, device=dev)
+            self._idx_free = None
         hp = self._pin.numpy()
         hp[:m] = plan.perm_src_local
         hp[m:2 * m] = plan.ret_idx
         hp[2 * m:need] = plan.local_offsets
+        if self._idx_free is not None:
+            torch.cuda.current_stream().wait_event(self._idx_free)
         self._idx[:need].copy_(self._pin[:need], non_blocking=True)
+        self._pin_copied = torch.cuda.Event()
+        self._pin_copied.record()
         perm_src_local, ret_idx, local_offsets = self._idx[:m], self._idx[m:2 * m], self._idx[2 * m:need]
 
         x_recv = torch.empty((max(n, 1), H), dtype=torch.bfloat16, device=dev)
@@ -167,6 +178,8 @@ class ExpertParallelMoE:
                            out_local.data_ptr(), ws.data_ptr(), ws.numel(), s)
             _lib.gather_rows(out_local.data_ptr(), n, H * 4, ret_idx.data_ptr(), 1, n, out_send.data_ptr(), s)
 
+        self._idx_free = torch.cuda.Event()
+        self._idx_free.record()                 # after the last kernel that reads _idx
         self.exchange.rows(L.out_perm, out_send[:n], plan.send_rows, plan.recv_rows)
         L.combine()
         return L.y
