@@ -33,10 +33,21 @@ def test_rotation_evicts_l2_between_visits(name):
 
 def test_workload_config_names_the_workload():
     w = inputs.WORKLOADS["decode_T64"]
-    cfg = bench.workload_config(w, 4, 512, 2, 124.5)
+    cfg = bench.workload_config(w, 4, 512, 2)
     assert cfg["workload"] == "decode_T64" and cfg["T"] == 64 and cfg["E"] == 128 and cfg["k"] == 8
     assert cfg["parallelism"] == "dp2 (independent batches)" and cfg["layers_rotated"] == 4
     assert "L2" in cfg["l2"]
+    # the config is a function of the workload and the run alone, so both arms print the same one
+    assert cfg == bench.workload_config(w, 4, 512, 2)
+
+
+def test_every_workload_family_is_reported():
+    names = set(bench.ALL_WORKLOADS)
+    assert {"tiny", "decode_T1", "decode_T8", "decode_T32", "decode_T64", "prefill_zipf_T4096", "slots512_T1",
+            "slots512_T2048", "slots512_T8192", "wide_T8192"} <= names
+    assert all(n in inputs.WORKLOADS for n in names)
+    assert bench.SWEEP_WORKLOAD == "wide_decode_T1" and inputs.WIDE_SWEEP_LAYERS == 48
+    assert bench.MEDIAN_REPLAYS >= 50
 
 
 def test_e2e_pipeline_with_no_steps_only_gates_the_copy_streams():
