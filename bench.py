@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: the experts split over the ranks, rows exchanged all-to-all "
                          "(each rank still brings its own tokens: weak scaling)")
+    ap.add_argument("--whole", action="store_true",
+                    help="run each layer through ft_moe_layer_nvfp4 (one launch for decode-sized batches)")
     ap.add_argument("--fused-front", action="store_true",
                     help="route and permute through ft_moe_route_permute (one launch for small batches)")
     ap.add_argument("--slot-churn", nargs="?", const="decode", default=None, choices=["decode", "prefill_stream"],
@@ -277,8 +279,10 @@ class E2EPipeline:
 
 def run_config(args, base: dict) -> dict:
     """The reported config: the workload's, plus the options that change what runs."""
-    return dict(base, format=args.fmt, slot_layout=args.layout,
-                front="ft_moe_route_permute" if args.fused_front else "ft_moe_route + ft_moe_permute")
+    calls = ("ft_moe_layer_nvfp4" if getattr(args, "whole", False) else
+             ("ft_moe_route_permute" if args.fused_front else "ft_moe_route + ft_moe_permute")
+             + " + ft_moe_ffn_nvfp4 + ft_moe_combine")
+    return dict(base, format=args.fmt, slot_layout=args.layout, calls=calls)
 
 
 # Workloads reported in the `workloads` object of the JSON line, besides the
@@ -408,7 +412,8 @@ def measure_workload(args, name, rank, world, local, dev, peaks, headline, want_
         lg = torch.from_numpy(li.logits).to(dev)
         layers.append(dict(li=li, pool=pool, st_host=st, st=torch.from_numpy(st).to(dev), x=x, lg=lg, seed=s))
     torch.cuda.synchronize()
-    layer = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev, fused_front=args.fused_front)
+    layer = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev, fused_front=args.fused_front,
+                     whole=args.whole)
     stream = torch.cuda.Stream(device=dev)
     tm = Timer(stream, world, dev)
 
@@ -466,7 +471,7 @@ def measure_workload(args, name, rank, world, local, dev, peaks, headline, want_
     bufs = []
     for _ in range(2):
         bufs.append(dict(lay=MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev,
-                                      fused_front=args.fused_front),
+                                      fused_front=args.fused_front, whole=args.whole),
                          xd=torch.empty_like(layers[0]["x"]), lgd=torch.empty_like(layers[0]["lg"]),
                          y_host=torch.empty((T, w.H), dtype=torch.float32).pin_memory()))
     e2e_graphs = {}
@@ -604,7 +609,7 @@ def measure_sweep(args, rank, world, local, dev, peaks, want_cpu):
                            x=torch.from_numpy(li.x_bits.view(np.int16)).view(torch.bfloat16).to(dev),
                            lg=torch.from_numpy(li.logits).to(dev),
                            lay=MoELayer(w.T, w.E, w.k, w.H, w.I, mode=w.route_mode, device=dev,
-                                        fused_front=args.fused_front)))
+                                        fused_front=args.fused_front, whole=args.whole)))
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
     tm = Timer(stream, world, dev)

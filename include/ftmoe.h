@@ -222,10 +222,11 @@ FT_API int ft_moe_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
  * f16:
  *   - every E2M1*E4M3 product is exact in f16;
  *   - each token row x_t is converted once, times the power of two 2^(12-e)
- *     that puts its largest magnitude in [2^14, 2^15) (e: max|x_t| * 2^-e in
- *     [4, 8); any finite bf16 row has one).  Elements within a factor 2^31 of
- *     the row's largest magnitude convert exactly; smaller ones round with an
- *     absolute error of at most 2^-39 max|x_t|;
+ *     that puts its largest magnitude in [2^13, 2^15) (e = 0 when max|x_t| is
+ *     in [2, 8), else max|x_t| * 2^-e is in [4, 8); any finite bf16 row has
+ *     one).  Elements within a factor 2^30 of the row's largest magnitude
+ *     convert exactly; smaller ones round with an absolute error of at most
+ *     2^-38 max|x_t|;
  *   - h is rounded to f16 after dividing it by 2^(2e), the square of its
  *     row's factor (undone exactly, in fp32, on the down projection's
  *     output), so its range does not depend on the row's magnitude, only
@@ -260,6 +261,40 @@ FT_API size_t ft_moe_ffn_workspace_size(int T, int H, int I, int E, int k);
  */
 FT_API int ft_moe_combine(const void* out_perm, const int32_t* pair_to_row, const float* topk_w,
                    int T, int k, int H, void* y, ft_stream_t stream);
+
+/*
+ * The whole layer -- route, permute, experts, combine -- as one call, with
+ * the outputs of the four calls above, bit for bit:
+ *   ft_moe_route(logits, T, E, k, mode, topk_ids, topk_w)
+ *   ft_moe_permute(topk_ids, T, k, E, expert_offsets, perm_src, pair_to_row)
+ *   ft_moe_ffn_nvfp4(x, T, H, I, E, k, perm_src, expert_offsets, slot_table, slot_pool, layout, out_perm)
+ *   ft_moe_combine(out_perm, pair_to_row, topk_w, T, k, H, y)
+ * (the steps of the layer as the pages' serving engine runs it: top-k router,
+ * grouping of the tokens per expert, NVFP4 expert FFNs, weighted sum;
+ * "FlashML-org / FreeToken" About page, "Fast Edge-Native Runtime", and the
+ * FreeToken model guide's MoE expert scheduling section).
+ *
+ * Decode-sized batches (few token rows per expert, T <= 128, T*k <= 1024,
+ * E <= 512) run all of it in ONE persistent kernel launch: the grid routes
+ * the tokens, every CTA sorts the pairs in its own shared memory, the expert
+ * GEMMs stream the weights as ft_moe_ffn_nvfp4 does, and the combine runs
+ * inside the down GEMM's epilogue.  Other sizes make the four calls.
+ *
+ * Arguments are those of the four calls (same layouts, same alignment
+ * rules); x bf16 [T, H], logits fp32 [T, E], y fp32 [T, H].
+ *   ws   device workspace of ft_moe_layer_workspace_size bytes, 256-B aligned.
+ *        It must be zero-filled once before its first use (cudaMemset); each
+ *        call leaves it ready for the next, including a call that recorded a
+ *        device status.  One workspace serves one call at a time.
+ * A token whose experts include a non-resident one (slot -1) gets no y row
+ * (FT_DEV_NOT_RESIDENT is recorded).
+ */
+FT_API int ft_moe_layer_nvfp4(const void* x, const float* logits, int T, int H, int I, int E, int k, int mode,
+                              const int32_t* slot_table, const void* slot_pool,
+                              const ft_nvfp4_slot_layout* layout, int32_t* topk_ids, float* topk_w,
+                              int32_t* expert_offsets, int32_t* perm_src, int32_t* pair_to_row, void* out_perm,
+                              void* y, void* ws, size_t ws_bytes, ft_stream_t stream);
+FT_API size_t ft_moe_layer_workspace_size(int T, int H, int I, int E, int k);
 
 /*
  * NVFP4 pack of one fp32 tensor [N, K] (K % 16 == 0), every step an IEEE fp32
@@ -452,7 +487,8 @@ enum {
   FT_KERNEL_FFN_DECODE = 8,   /* decode variant: gate/up + SwiGLU + down in one launch */
   FT_KERNEL_GATHER = 9,       /* row gather of the expert-parallel exchange */
   FT_KERNEL_ROUTE_PERMUTE = 10, /* route and permute in one launch (small batches) */
-  FT_KERNEL_KINDS = 11,
+  FT_KERNEL_LAYER_DECODE = 11,  /* the whole layer in one launch (ft_moe_layer_nvfp4, small batches) */
+  FT_KERNEL_KINDS = 12,
 };
 
 typedef struct {

@@ -54,7 +54,7 @@ class SlotLayout(ctypes.Structure):
 
 
 FT_KERNEL_NAMES = ("route", "permute", "schedule", "gemm_gate_up", "gemm_down", "combine", "pack", "prep_x",
-                   "ffn_decode", "gather", "route_permute")
+                   "ffn_decode", "gather", "route_permute", "layer_decode")
 
 
 class Profile(ctypes.Structure):
@@ -82,6 +82,10 @@ _SIGS = {
                                  c_void_p, POINTER(SlotLayout), c_void_p, c_void_p, c_size_t, c_void_p]),
     "ft_moe_ffn_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "ft_moe_combine": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
+    "ft_moe_layer_nvfp4": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p,
+                                   POINTER(SlotLayout), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   c_void_p, c_void_p, c_size_t, c_void_p]),
+    "ft_moe_layer_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "ft_nvfp4_pack": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "ft_mxfp4_pack": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "ft_device_status": (c_int, [POINTER(c_int), c_int]),
@@ -177,6 +181,16 @@ def ffn_nvfp4(x, T, H, I, E, k, perm_src, offsets, slot_table, pool, layout, out
 
 def combine(out_perm, pair_to_row, w, T, k, H, y, stream) -> None:
     check(lib().ft_moe_combine(out_perm, pair_to_row, w, T, k, H, y, stream))
+
+
+def layer_workspace_size(T, H, I, E, k) -> int:
+    return int(lib().ft_moe_layer_workspace_size(T, H, I, E, k))
+
+
+def layer_nvfp4(x, logits, T, H, I, E, k, mode, slot_table, pool, layout, ids, w, offsets, perm_src, pair_to_row,
+                out_perm, y, ws, ws_bytes, stream) -> None:
+    check(lib().ft_moe_layer_nvfp4(x, logits, T, H, I, E, k, mode, slot_table, pool, ctypes.byref(layout), ids, w,
+                                   offsets, perm_src, pair_to_row, out_perm, y, ws, ws_bytes, stream))
 
 
 def gather_rows(src, n_src, row_bytes, idx, div, n, dst, stream) -> None:

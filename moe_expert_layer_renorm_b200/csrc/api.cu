@@ -203,6 +203,45 @@ extern "C" int ft_moe_combine(const void* out_perm, const int32_t* pair_to_row, 
   return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_combine");
 }
 
+extern "C" size_t ft_moe_layer_workspace_size(int T, int H, int I, int E, int k) {
+  if (T <= 0 || !ffn_shape_ok(H, I, E, k)) return 0;
+  return plan_layer(T, H, I, E, k, device_sm_count()).total;
+}
+
+extern "C" int ft_moe_layer_nvfp4(const void* x, const float* logits, int T, int H, int I, int E, int k, int mode,
+                                  const int32_t* slot_table, const void* slot_pool,
+                                  const ft_nvfp4_slot_layout* layout, int32_t* ids, float* w, int32_t* offsets,
+                                  int32_t* perm_src, int32_t* pair_to_row, void* out_perm, void* y, void* ws,
+                                  size_t ws_bytes, ft_stream_t stream) {
+  if (T < 0 || !ffn_shape_ok(H, I, E, k) || k > 32 || (mode != FT_ROUTE_SOFTMAX_RENORM && mode != FT_ROUTE_TOPK_SOFTMAX))
+    return fail(FT_ERR_UNSUPPORTED,
+                "ft_moe_layer_nvfp4: need H, I >= 256 and multiples of 64, 1 <= k <= min(E, 32), E <= 1024, a mode");
+  if (!offsets) return fail(FT_ERR_INVALID_ARG, "ft_moe_layer_nvfp4: null pointer");
+  const cudaStream_t s = S(stream);
+  if (T == 0) {
+    const cudaError_t e = cudaMemsetAsync(offsets, 0, size_t(E + 1) * sizeof(int32_t), s);
+    return e == cudaSuccess ? FT_OK : cuda_fail(e, "ft_moe_layer_nvfp4");
+  }
+  if (!x || !logits || !slot_table || !slot_pool || !layout || !ids || !w || !perm_src || !pair_to_row ||
+      !out_perm || !y || !ws)
+    return fail(FT_ERR_INVALID_ARG, "ft_moe_layer_nvfp4: null pointer");
+  if (layout->H != H || layout->I != I || layout->num_slots < 1 || layout->num_slots > (1 << 21) ||
+      (layout->tiled != 0 && layout->tiled != 1) || layout->slot_bytes % 256 ||
+      (layout->scale_format != FT_SCALE_NVFP4 && layout->scale_format != FT_SCALE_MXFP4))
+    return fail(FT_ERR_INVALID_ARG,
+                "ft_moe_layer_nvfp4: layout does not match H, I (or has more than 2^21 slots, or an unknown format)");
+  if ((reinterpret_cast<uintptr_t>(slot_pool) & 255) || (reinterpret_cast<uintptr_t>(ws) & 255) ||
+      (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(out_perm) & 15) ||
+      (reinterpret_cast<uintptr_t>(y) & 15))
+    return fail(FT_ERR_INVALID_ARG, "ft_moe_layer_nvfp4: misaligned pointer");
+  if (ws_bytes < plan_layer(T, H, I, E, k, device_sm_count()).total)
+    return fail(FT_ERR_INVALID_ARG, "ft_moe_layer_nvfp4: workspace too small");
+  const char* why = "ft_moe_layer_nvfp4";
+  const cudaError_t e = launch_layer(x, logits, T, H, I, E, k, mode, slot_table, slot_pool, *layout, ids, w, offsets,
+                                     perm_src, pair_to_row, out_perm, y, ws, s, &why);
+  return e == cudaSuccess ? FT_OK : cuda_fail(e, why);
+}
+
 extern "C" int ft_gather_rows(const void* src, int n_src, int row_bytes, const int32_t* idx, int div, int n,
                               void* dst, ft_stream_t stream) {
   if (n < 0 || n_src < 0 || row_bytes < 16 || row_bytes % 16 || div < 1)

@@ -223,6 +223,7 @@ __device__ __forceinline__ bool dec_epilogue(const DecodeParams& p, const DecUni
     if (lane == 0) last = atom_acq_rel_gpu_add(G.counters + (d.u / G.splits) * 16 + w, 1) == G.splits - 1;
     last = __shfl_sync(0xFFFFFFFFu, last, 0);
     if (!last) return false;
+    if (lane == 0) G.counters[(d.u / G.splits) * 16 + w] = 0;   // every split has arrived: ready for the next call
     const int u0 = d.u - d.split;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {

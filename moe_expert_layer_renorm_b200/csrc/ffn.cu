@@ -29,6 +29,8 @@
 // Every pipeline wait is bounded (see sm100.cuh); a wait that gives up sets
 // the device status word and an abort flag, all roles leave their loops, and
 // the CTA drains its outstanding copies and MMAs before freeing tensor memory.
+#include <type_traits>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -190,16 +192,18 @@ struct Abort {
 };
 
 // Per-row normalisation of the token rows.  Row r (token t) has the
-// exponent e_r with max|x_t| * 2^-e_r in [4, 8) (e_r = 0 for an all-zero row),
-// and rowscale[r] = f_r = 2^e_r.  GEMM1 multiplies f16 operands
-// x' = x * 2^(12 - e_r) (largest magnitude in [2^14, 2^15)), so with the
-// global scale gG its accumulator gives G' = gG * 2^-12 * acc = G / f_r: the
-// gate (and likewise the up) projection of the row scaled to a largest
-// magnitude in [4, 8).  h is stored normalised the same way,
+// exponent e_r (row_exp_of_max: 0 when max|x_t| is in [2, 8), else
+// max|x_t| * 2^-e_r in [4, 8)), and rowscale[r] = f_r = 2^e_r.  GEMM1
+// multiplies f16 operands x' = x * 2^(12 - e_r) (largest magnitude in
+// [2^13, 2^15)), so with the global scale gG its accumulator gives
+// G' = gG * 2^-12 * acc = G / f_r: the gate (and likewise the up) projection
+// of the row scaled to a largest magnitude in [2, 8).  h is stored normalised
+// the same way,
 //   h' = silu(G) * U / f_r^2 = G' * U' / (1 + e^-(G' f_r)),
 // so its f16 range does not depend on the row's magnitude, and GEMM2 undoes
-// it exactly: out = (gD * acc * f_r) * f_r.  For rows of largest magnitude in
-// [4, 8) (the N(0, 1) workloads) f_r = 1 and nothing changes.
+// it exactly: out = (gD * acc * f_r) * f_r.  Rows of ordinary magnitude (the
+// N(0, 1) workloads) have f_r = 1, and the epilogues skip the factor for
+// units whose rows all have it.
 constexpr float kRowNormInv = 1.0f / 4096.0f;   // 2^-12
 
 // h' = g * u / (1 + e^-(g f)).  The hardware exponential and a fast divide: a
@@ -208,6 +212,8 @@ constexpr float kRowNormInv = 1.0f / 4096.0f;   // 2^-12
 __device__ __forceinline__ float silu_mul(float g, float u, float f) {
   return __fdividef(g * u, 1.0f + __expf(-(g * f)));
 }
+// The same for f = 1.
+__device__ __forceinline__ float silu_mul1(float g, float u) { return __fdividef(g * u, 1.0f + __expf(-g)); }
 // GEMM2's output from its accumulator: (gD * acc * f) * f, in this order so
 // that no intermediate leaves the fp32 range when the result does not.
 __device__ __forceinline__ float down_out(float gd, float acc, float f) { return (gd * acc * f) * f; }
@@ -522,41 +528,55 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
         for (int m = 0; m < NMAT; ++m) tmem_ld_32x32b_x16(dcol + m * BN, v[0][m]);
       }
       bool released = false;
+      // Two versions of the block loop: rows whose factors are all 1 (every
+      // row of activations of ordinary magnitude) skip the per-row factor --
+      // a broadcast and two multiplies per element, which in the down GEMM's
+      // epilogue are as long as the unit's MMAs.  The test is warp-uniform.
+      bool unit_scaled = false;
 #pragma unroll
-      for (int bk = 0; bk < BN / 16; ++bk) {
-        const int n0 = bk * 16;
-        if (n0 >= n_eff) break;
-        tmem_wait_ld();
-        if (n0 + 16 < n_eff) {
+      for (int g = 0; g < kGroups; ++g) unit_scaled |= tsl[g] != 1.0f;
+      unit_scaled = __any_sync(0xFFFFFFFFu, unit_scaled);
+      auto blocks = [&](auto scaled_tag) {
+        constexpr bool kScaled = decltype(scaled_tag)::value;
 #pragma unroll
-          for (int m = 0; m < NMAT; ++m) tmem_ld_32x32b_x16(dcol + m * BN + n0 + 16, v[(bk + 1) & 1][m]);
-        } else {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&d_empty[ds]);
-          released = true;
-        }
-        const uint32_t (&w)[NMAT][16] = v[bk & 1];
+        for (int bk = 0; bk < BN / 16; ++bk) {
+          const int n0 = bk * 16;
+          if (n0 >= n_eff) break;
+          tmem_wait_ld();
+          if (n0 + 16 < n_eff) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int n = n0 + i;
-          const float ts = __shfl_sync(0xFFFFFFFFu, tsl[bk >> 1], (bk & 1) * 16 + i);
-          if (n >= nr) break;
-          if (split) {
+            for (int m = 0; m < NMAT; ++m) tmem_ld_32x32b_x16(dcol + m * BN + n0 + 16, v[(bk + 1) & 1][m]);
+          } else {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[ds]);
+            released = true;
+          }
+          const uint32_t (&w)[NMAT][16] = v[bk & 1];
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m)
-              p.partials[(size_t(u) * NMAT + m) * 128 * BN + size_t(n) * 128 + row] = __uint_as_float(w[m][i]);
-          } else if (feat < p.M) {
-            float r;
-            if (NMAT == 2) {
-              r = silu_mul(gsc[0] * __uint_as_float(w[0][i]), gsc[NMAT - 1] * __uint_as_float(w[NMAT - 1][i]), ts);
-            } else {
-              r = down_out(gsc[0], __uint_as_float(w[0][i]), ts);
+          for (int i = 0; i < 16; ++i) {
+            const int n = n0 + i;
+            const float ts = kScaled ? __shfl_sync(0xFFFFFFFFu, tsl[bk >> 1], (bk & 1) * 16 + i) : 1.0f;
+            if (n >= nr) break;
+            if (split) {
+#pragma unroll
+              for (int m = 0; m < NMAT; ++m)
+                p.partials[(size_t(u) * NMAT + m) * 128 * BN + size_t(n) * 128 + row] = __uint_as_float(w[m][i]);
+            } else if (feat < p.M) {
+              float r;
+              if (NMAT == 2) {
+                r = kScaled ? silu_mul(gsc[0] * __uint_as_float(w[0][i]), gsc[NMAT - 1] * __uint_as_float(w[NMAT - 1][i]), ts)
+                            : silu_mul1(gsc[0] * __uint_as_float(w[0][i]), gsc[NMAT - 1] * __uint_as_float(w[NMAT - 1][i]));
+              } else {
+                r = kScaled ? down_out(gsc[0], __uint_as_float(w[0][i]), ts) : gsc[0] * __uint_as_float(w[0][i]);
+              }
+              store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
             }
-            store_out<NMAT>(p.out, size_t(rb + n) * p.M + feat, r);
           }
         }
-      }
+      };
+      if (unit_scaled) blocks(std::true_type{});
+      else blocks(std::false_type{});
       if (!released) {
         tc_fence_before();
         __syncwarp();
@@ -729,9 +749,18 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& v, float fa, float
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// The row exponent e_r from the row's largest magnitude m (warp-wide max
-// first): m * 2^-e_r in [4, 8); 0 for an all-zero row, and for a non-finite
-// one, which also records FT_DEV_F16_RANGE.
+// The row exponent e_r of a row whose largest magnitude is m (finite):
+// 0 when m is in [2, 8) (rows of ordinary magnitude keep the factor 1) or
+// m = 0, else the e_r with m * 2^-e_r in [4, 8).
+__device__ __forceinline__ int row_exp_of_max(float m) {
+  if (m == 0.0f || (m >= 2.0f && m < 8.0f)) return 0;
+  int e;
+  frexpf(m, &e);                                 // m = f * 2^e, f in [0.5, 1); exact for subnormals too
+  return e - 3;                                  // m * 2^-(e - 3) = 8 f in [4, 8)
+}
+
+// The row exponent from the row's largest magnitude (warp-wide max first); 0
+// for a non-finite row, which also records FT_DEV_F16_RANGE.
 __device__ __forceinline__ int prep_row_exp(float m) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
@@ -739,21 +768,17 @@ __device__ __forceinline__ int prep_row_exp(float m) {
     set_device_status(FT_DEV_F16_RANGE);         // inf or nan input
     return 0;
   }
-  if (m == 0.0f) return 0;
-  int e;
-  frexpf(m, &e);                                 // m = f * 2^e, f in [0.5, 1); exact for subnormals too
-  return e - 3;                                  // m * 2^-(e - 3) = 8 f in [4, 8)
+  return row_exp_of_max(m);
 }
 
 // One warp per permuted row r (token t = perm_src[r] / k): writes
 // x_perm[r] = f16(x[t] * 2^(12 - e_r)) and rowscale[r] = 2^e_r, e_r the row
-// exponent (max|x[t]| * 2^-e_r in [4, 8), so the converted row's largest
-// magnitude is in [2^14, 2^15)).  Every finite bf16 row qualifies (e_r in
-// [-135, 125]).  The f16 conversion is exact for every element of the row
-// within a factor 2^31 of the row's largest magnitude (bf16 has 8
-// significant bits; f16 represents those exactly down to 2^-17); smaller
-// elements round, to f16 subnormals, with an absolute error of at most
-// 2^-25 in converted units, below 2^-39 max|x[t]|.
+// exponent (so the converted row's largest magnitude is in [2^13, 2^15)).
+// Every finite bf16 row qualifies (e_r in [-135, 125]).  The f16 conversion
+// is exact for every element of the row within a factor 2^30 of the row's
+// largest magnitude (bf16 has 8 significant bits; f16 represents those
+// exactly down to 2^-17); smaller elements round, to f16 subnormals, with an
+// absolute error of at most 2^-25 in converted units, below 2^-38 max|x[t]|.
 // Rows in permuted order make each expert group's tokens one contiguous
 // block, so the GEMM loads them as plain tiles.  Rows of up to 3072 values
 // are read once into registers with all loads in flight together (the

@@ -16,6 +16,7 @@
 #include "decode.cu"
 #include "selftest.cu"
 #include "ffn_host.cu"
+#include "layer.cu"
 #include "api.cu"
 #include "permute_noalloc.cu"
 #include "slots.cpp"

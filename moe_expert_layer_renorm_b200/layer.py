@@ -104,9 +104,11 @@ class MoELayer:
     """Buffers and calls for one MoE FFN layer of fixed (T, E, k, H, I)."""
 
     def __init__(self, T: int, E: int, k: int, H: int, I: int, mode: int = _lib.FT_ROUTE_SOFTMAX_RENORM,
-                 device="cuda", fused_front: bool = False):
+                 device="cuda", fused_front: bool = False, whole: bool = False):
         self.T, self.E, self.k, self.H, self.I, self.mode = T, E, k, H, I, mode
-        self.fused_front = fused_front   # route + permute through ft_moe_route_permute
+        self.fused_front = fused_front   # route + permute through ft_moe_route_permute (separate calls only)
+        # forward() through ft_moe_layer_nvfp4 (one launch for decode-sized batches); False: the four calls
+        self.whole = whole and not fused_front
         P = T * k
         dev = torch.device(device)
         i32 = dict(dtype=torch.int32, device=dev)
@@ -117,10 +119,31 @@ class MoELayer:
         self.pair_to_row = torch.empty(P, **i32)
         self.out_perm = torch.empty((P, H), dtype=torch.float32, device=dev)
         self.y = torch.empty((T, H), dtype=torch.float32, device=dev)
+        self.dev = dev
         self.perm_ws_bytes = _lib.permute_workspace_size(T, k, E)
-        self.perm_ws = torch.empty(max(self.perm_ws_bytes, 256), dtype=torch.uint8, device=dev)
         self.ffn_ws_bytes = _lib.ffn_workspace_size(T, H, I, E, k)
-        self.ffn_ws = torch.empty(max(self.ffn_ws_bytes, 256), dtype=torch.uint8, device=dev)
+        self.layer_ws_bytes = _lib.layer_workspace_size(T, H, I, E, k)
+        self._perm_ws = self._ffn_ws = self._layer_ws = None
+
+    # workspaces, allocated on first use: the separate calls' (permute, ffn) and
+    # the whole-layer call's, which is zero-filled once and left ready by every call
+    @property
+    def perm_ws(self) -> torch.Tensor:
+        if self._perm_ws is None:
+            self._perm_ws = torch.empty(max(self.perm_ws_bytes, 256), dtype=torch.uint8, device=self.dev)
+        return self._perm_ws
+
+    @property
+    def ffn_ws(self) -> torch.Tensor:
+        if self._ffn_ws is None:
+            self._ffn_ws = torch.empty(max(self.ffn_ws_bytes, 256), dtype=torch.uint8, device=self.dev)
+        return self._ffn_ws
+
+    @property
+    def layer_ws(self) -> torch.Tensor:
+        if self._layer_ws is None:
+            self._layer_ws = torch.zeros(max(self.layer_ws_bytes, 256), dtype=torch.uint8, device=self.dev)
+        return self._layer_ws
 
     def route(self, logits: torch.Tensor, stream=None) -> None:
         _lib.route(logits.data_ptr(), self.T, self.E, self.k, self.mode, self.ids.data_ptr(), self.w.data_ptr(),
@@ -144,12 +167,24 @@ class MoELayer:
         _lib.combine(self.out_perm.data_ptr(), self.pair_to_row.data_ptr(), self.w.data_ptr(), self.T, self.k,
                      self.H, self.y.data_ptr(), _stream(stream))
 
+    def layer(self, x: torch.Tensor, logits: torch.Tensor, slot_table: torch.Tensor, pool: ExpertPool,
+              stream=None) -> None:
+        _lib.layer_nvfp4(x.data_ptr(), logits.data_ptr(), self.T, self.H, self.I, self.E, self.k, self.mode,
+                         slot_table.data_ptr(), pool.ptr, pool.layout, self.ids.data_ptr(), self.w.data_ptr(),
+                         self.offsets.data_ptr(), self.perm_src.data_ptr(), self.pair_to_row.data_ptr(),
+                         self.out_perm.data_ptr(), self.y.data_ptr(), self.layer_ws.data_ptr(), self.layer_ws_bytes,
+                         _stream(stream))
+
     def forward(self, x: torch.Tensor, logits: torch.Tensor, slot_table: torch.Tensor, pool: ExpertPool,
                 stream=None) -> torch.Tensor:
-        """route -> permute -> ffn -> combine, enqueued on one stream."""
+        """route -> permute -> ffn -> combine, enqueued on one stream (one ft_moe_layer_nvfp4 call, or
+        the four calls when the layer was made with whole=False)."""
         assert x.dtype == torch.bfloat16 and x.shape == (self.T, self.H) and x.is_contiguous()
         assert logits.dtype == torch.float32 and logits.shape == (self.T, self.E) and logits.is_contiguous()
         assert slot_table.dtype == torch.int32 and slot_table.numel() == self.E
+        if self.whole:
+            self.layer(x, logits, slot_table, pool, stream)
+            return self.y
         if self.fused_front:
             self.route_permute(logits, stream)
         else:

@@ -53,8 +53,29 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
+def _a256(n: int) -> int:
+    return (n + 255) // 256 * 256
+
+
+def poison(lay: MoELayer) -> None:
+    """Fill what the layer writes before it reads with NaN (0xFF bytes): the
+    outputs, the separate calls' FFN workspace, and the data part of the
+    whole-layer workspace (its f16 token rows, row factors and h, which come
+    before its counters; the counters must stay zero)."""
+    lay.out_perm.fill_(float("nan"))
+    lay.y.fill_(float("nan"))
+    if lay.whole:
+        T, k, H, I = lay.T, lay.k, lay.H, lay.I
+        data = _a256(T * H * 2) + _a256(T * 4) + _a256(T * k * I * 2)
+        ws = lay.layer_ws
+        ws[:min(data, ws.numel())].fill_(0xFF)
+    else:
+        lay.ffn_ws.fill_(0xFF)
+
+
 def run_gpu(w: inputs.Workload, T: Optional[int] = None, layer: int = 0, pool=None, slot_table=None,
-            li: Optional[inputs.LayerInputs] = None, expect_status: int = 0, fused_front: bool = False) -> GpuRun:
+            li: Optional[inputs.LayerInputs] = None, expect_status: int = 0, fused_front: bool = False,
+            whole: bool = False) -> GpuRun:
     li = li or inputs.make_layer_inputs(w, layer, T)
     T = li.x_bits.shape[0]
     if pool is None:
@@ -62,11 +83,10 @@ def run_gpu(w: inputs.Workload, T: Optional[int] = None, layer: int = 0, pool=No
     x = torch.from_numpy(li.x_bits.view(np.int16)).view(torch.bfloat16).cuda()
     logits = torch.from_numpy(li.logits).cuda()
     st = torch.from_numpy(np.asarray(slot_table, dtype=np.int32)).cuda()
-    lay = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, fused_front=fused_front)
+    lay = MoELayer(T, w.E, w.k, w.H, w.I, mode=w.route_mode, fused_front=fused_front, whole=whole)
     # NaN in every intermediate the library writes before reading: an element
     # read before it is written (a missed dependency) shows up in y
-    lay.ffn_ws.fill_(0xFF)
-    lay.out_perm.fill_(float("nan"))
+    poison(lay)
     from moe_expert_layer_renorm_b200 import _lib
     _lib.device_status(clear=True)
     y = lay.forward(x, logits, st, pool)
