@@ -31,16 +31,14 @@
 //            unit are gathered from the token-ordered f16 copy by cp.async
 //            (row r of the tile is token perm_src[r] / k) instead of a TMA box
 //            of a permuted copy; down units read h by TMA as before.
-//   phase 4  combine, fused into the down epilogue: each compute warp owns 16
-//            output features of a 256-row tile; after storing them for its
-//            rows it adds one to a counter per (token, tile, warp) (release).
-//            The warp that brings a token's counter to k -- all k expert
-//            outputs of those features are then in place -- sums them in the
-//            order j = 0 .. k-1 with the combine kernel's arithmetic, so y is
-//            bit-identical to ft_moe_combine's.
+//   phase 4  combine: each CTA publishes how many down units it finished
+//            (one release after its last unit); once the count reaches the
+//            number of down units, every CTA sums a strided share of the
+//            output vectors in the order j = 0 .. k-1 with the combine
+//            kernel's arithmetic, so y is bit-identical to ft_moe_combine's.
 //
-// Workspace counters (routed tokens, the unit queue, CTAs done, h published
-// per token tile, split-K arrivals, combine arrivals) start at zero: the
+// Workspace counters (routed tokens, converted rows, the unit queue, down
+// units done, CTAs done, h published per token tile, split-K arrivals) start at zero: the
 // caller zero-fills the workspace once, and every call leaves them at zero
 // again (each counter is reset by the last thread to use it; the last CTA to
 // finish resets the rest, and everything after a call that recorded a device
@@ -62,6 +60,8 @@ static_assert(kLayerSmemBytes <= 227 * 1024, "shared memory budget");
 // Barrier tags of the waits for every token to be routed / every row converted.
 constexpr int kTagRouted = 11;
 constexpr int kTagConverted = 12;
+constexpr int kTagCombine = 13;    // the wait for every down unit before the combine
+constexpr int kLayerCtrl = 6;      // control counters in the workspace
 
 struct LayerParams {
   DecodeParams d;              // the FFN steps; d.g[*].units are unused (units come from the sort)
@@ -77,8 +77,7 @@ struct LayerParams {
   uint4* x16;                  // [T, H] f16, token order (workspace)
   float* rowscale;             // [T] row factors 2^e_t (workspace)
   int* ctrl;                   // [0] tokens routed, [1] unit queue, [2] CTAs done, [3] phase-1 items claimed,
-                               // [4] rows converted (workspace)
-  int* ccnt;                   // [T][mt2][16] combine arrivals (workspace)
+                               // [4] rows converted, [5] down units done (workspace)
   int* tile_done;              // per token tile: h rows published (workspace)
   int* cnt1;                   // split-K arrivals of gate/up, n_cnt1 ints
   int* cnt2;                   // split-K arrivals of down, n_cnt2 ints
@@ -101,7 +100,8 @@ struct LayerTables {
                   // [kMiscConv] the wait for converted rows gave up
 };
 constexpr int kMiscClaim = 36;
-constexpr int kMiscConv = 37;
+constexpr int kMiscConv = 37;      // a wait of phase 2b or 4 gave up
+constexpr int kMiscDown = 38;      // down units this CTA finished
 // Named barrier of the warps that run phase 2b (all but the weight producer).
 constexpr int kBarPhase2 = 1;
 
@@ -337,9 +337,8 @@ __device__ __forceinline__ void layer_gather_stage(const LayerParams& p, const G
   cp_async_mbar_arrive_noinc(bar);
 }
 
-// Compute warp w's part of one unit (the decode kernel's dec_unit with the
-// row factors from the shared-memory tables and the combine after the down
-// epilogue).
+// Compute warp w's part of one unit: the decode kernel's dec_unit with the
+// row factors from the shared-memory tables.
 template <int NT, int FMT>
 __device__ bool layer_unit(const LayerParams& p, const LayerTables& tb, const DecUnit& d, uint8_t* smem,
                            uint64_t* full, uint64_t* empty, const Abort& ab, uint64_t* unit_free,
@@ -390,57 +389,7 @@ __device__ bool layer_unit(const LayerParams& p, const LayerTables& tb, const De
     mbar_arrive(&hpub[gu & 1]);
     return true;
   }
-  if (!fin) return true;
-  // combine: this warp's 16 features (mt * 256 + 16 w .. + 15) of each of its
-  // rows are stored; count them per token, and the k-th arrival sums them
-  __threadfence();
-  __syncwarp();
-  const int k = p.k;
-  int tok = -1, last = 0;
-  if (lane < d.nr) {
-    tok = tb.ps[d.rb + lane] / k;
-    last = atom_acq_rel_gpu_add(p.ccnt + (size_t(tok) * dp.mt2 + d.mt) * 16 + w, 1) == k - 1;
-  }
-  uint32_t todo = __ballot_sync(0xFFFFFFFFu, last);
-  const float* op = static_cast<const float*>(dp.g[1].out);
-  const int P = p.T * k;
-  const int f = d.mt * kDecRows + 16 * w + (lane & 15);
-  while (todo) {
-    // half-warp hw takes the next token of the list (two tokens per pass)
-    const int src0 = __ffs(todo) - 1;
-    todo &= todo - 1;
-    const int src1 = todo ? __ffs(todo) - 1 : -1;
-    if (src1 >= 0) todo &= todo - 1;
-    const int t0 = __shfl_sync(0xFFFFFFFFu, tok, src0);
-    const int t1 = __shfl_sync(0xFFFFFFFFu, tok, src1 < 0 ? src0 : src1);
-    const int tt = lane < 16 ? t0 : t1;
-    if ((lane < 16 || src1 >= 0) && f < p.H) {
-      // the order and arithmetic of the combine kernel: fmaf in j order,
-      // with each batch's rows and weights requested before they are used
-      float s = 0.0f;
-      for (int j0 = 0; j0 < k; j0 += 8) {
-        int row[8];
-        float wj[8], o[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          row[q] = j0 + q < k ? tb.p2r[tt * k + j0 + q] : -1;
-          wj[q] = j0 + q < k ? tb.w[tt * k + j0 + q] : 0.0f;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const bool ok = row[q] >= 0 && row[q] < P;
-          if (j0 + q < k && !ok) set_device_status(FT_DEV_BAD_INDEX);
-          o[q] = ok ? __ldcg(op + size_t(row[q]) * p.H + f) : 0.0f;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (row[q] >= 0 && row[q] < P) s = fmaf(wj[q], o[q], s);
-      }
-      p.y[size_t(tt) * p.H + f] = s;
-    }
-    if (lane == src0) p.ccnt[(size_t(t0) * dp.mt2 + d.mt) * 16 + w] = 0;
-    if (src1 >= 0 && lane == src1) p.ccnt[(size_t(t1) * dp.mt2 + d.mt) * 16 + w] = 0;
-  }
+  (void)fin;
   return true;
 }
 
@@ -472,6 +421,7 @@ layer_decode_kernel(const LayerParams p, const __grid_constant__ CUtensorMap tm_
     for (int i = 0; i < kDecUnitRing; ++i) { mbar_init(&ufull[i], 1); mbar_init(&uempty[i], 18); }
     for (int i = 0; i < 2; ++i) { mbar_init(&hpub[i], 512); hcount[i] = 0; }
     *abort_flag = 0;
+    tb.misc[kMiscDown] = 0;
     fence_mbarrier_init();
   }
   if (warp == 16 && lane == 0) {
@@ -501,7 +451,8 @@ layer_decode_kernel(const LayerParams p, const __grid_constant__ CUtensorMap tm_
     } else {
       layer_convert_row(p, item - p.T, reinterpret_cast<float*>(scratch));
     }
-    __threadfence();                 // this thread's ids and weights, or f16 row and factor
+    // the barrier orders every thread's writes before thread 0's release
+    // (cumulative at GPU scope), which publishes them with the count
     __syncthreads();
     if (threadIdx.x == 0) red_release_gpu_add(p.ctrl + (item < p.T ? 0 : 4), 1);
   }
@@ -646,6 +597,7 @@ layer_decode_kernel(const LayerParams p, const __grid_constant__ CUtensorMap tm_
       }
       const DecUnit d = decode_unit(p.d, q, n1, udesc[us]);
       const int gu = d.gemm == 0 ? ngu++ : -1;
+      if (d.gemm == 1 && warp == 0 && lane == 0) ++tb.misc[kMiscDown];
       const bool ok =
           d.nr > 8 ? layer_unit<2, FMT>(p, tb, d, smem, full, empty, ab, &uempty[us], &uent[us], hpub, hcount, gu, si, q, warp, lane)
                    : layer_unit<1, FMT>(p, tb, d, smem, full, empty, ab, &uempty[us], &uent[us], hpub, hcount, gu, si, q, warp, lane);
@@ -653,6 +605,59 @@ layer_decode_kernel(const LayerParams p, const __grid_constant__ CUtensorMap tm_
     }
   }
   __syncthreads();
+
+  // ------------------------------------------------------------ phase 4 ---
+  // The combine, once every down unit of the layer is done: this CTA's down
+  // units are published with one release (the barrier above orders all its
+  // threads' expert-output stores before it), then every CTA waits until the
+  // count reaches the number of down units and sums a strided share of the
+  // T x H/4 output vectors -- the combine kernel's arithmetic (fmaf in the
+  // order j = 0 .. k-1, each batch's rows and weights requested first), so y
+  // is the same bits.  Units are counted, not CTAs, so the wait never depends
+  // on a CTA that has not started.
+  if (counted && sorted) {
+    if (threadIdx.x == 0) {
+      red_release_gpu_add(p.ctrl + 5, tb.misc[kMiscDown]);
+      tb.misc[kMiscConv] = layer_wait_count(p.ctrl + 5, ntot - n1, kTagCombine) ? 0 : 1;
+    }
+    __syncthreads();
+    if (!tb.misc[kMiscConv]) {
+      const int k = p.k, vpr = p.H / 4, P = p.T * k;
+      const float4* op = static_cast<const float4*>(p.d.g[1].out);
+      float4* y = reinterpret_cast<float4*>(p.y);
+      const long long nvec = (long long)p.T * vpr;
+      for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nvec;
+           i += (long long)gridDim.x * blockDim.x) {
+        const int t = int(i / vpr), c = int(i % vpr);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j0 = 0; j0 < k; j0 += 4) {
+          int row[4];
+          float wj[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            row[q] = j0 + q < k ? tb.p2r[t * k + j0 + q] : -1;
+            wj[q] = j0 + q < k ? tb.w[t * k + j0 + q] : 0.0f;
+          }
+          float4 o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const bool ok = row[q] >= 0 && row[q] < P;
+            if (j0 + q < k && !ok) set_device_status(FT_DEV_BAD_INDEX);
+            o[q] = ok ? __ldcg(op + size_t(row[q]) * vpr + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (row[q] < 0 || row[q] >= P) continue;
+            acc.x = fmaf(wj[q], o[q].x, acc.x);
+            acc.y = fmaf(wj[q], o[q].y, acc.y);
+            acc.z = fmaf(wj[q], o[q].z, acc.z);
+            acc.w = fmaf(wj[q], o[q].w, acc.w);
+          }
+        }
+        y[i] = acc;
+      }
+    }
+  }
 
   // ------------------------------------------------ end: counter resets ---
   if (threadIdx.x == 0) {
@@ -665,12 +670,11 @@ layer_decode_kernel(const LayerParams p, const __grid_constant__ CUtensorMap tm_
     const int ntiles = dirty ? p.n_done : tb.misc[3];
     for (int i = threadIdx.x; i < ntiles; i += blockDim.x) p.d.tile_done[i] = 0;
     if (dirty) {
-      const int nc = p.T * p.d.mt2 * 16;
-      for (int i = threadIdx.x; i < nc; i += blockDim.x) p.ccnt[i] = 0;
       for (int i = threadIdx.x; i < p.n_cnt1; i += blockDim.x) p.cnt1[i] = 0;
       for (int i = threadIdx.x; i < p.n_cnt2; i += blockDim.x) p.cnt2[i] = 0;
     }
-    if (threadIdx.x == 0) { p.ctrl[0] = 0; p.ctrl[1] = 0; p.ctrl[2] = 0; p.ctrl[3] = 0; p.ctrl[4] = 0; }
+    if (threadIdx.x == 0)
+      for (int i = 0; i < kLayerCtrl; ++i) p.ctrl[i] = 0;
   }
 }
 
@@ -684,7 +688,7 @@ struct LayerPlan {
   bool fused;
   FfnPlan ffn;
   // fused: workspace layout (byte offsets)
-  size_t off_x16, off_rs, off_h, off_ctrl, off_ccnt, off_done, off_cnt1, off_cnt2, off_part1, off_part2;
+  size_t off_x16, off_rs, off_h, off_ctrl, off_done, off_cnt1, off_cnt2, off_part1, off_part2;
   int n_done, n_cnt1, n_cnt2;
   // separate calls: permute workspace, then the FFN workspace
   size_t off_perm_ws, off_ffn_ws;
@@ -706,8 +710,7 @@ static LayerPlan plan_layer(int T, int H, int I, int E, int k, int num_sms) {
     L.off_x16 = o;   o = align256(o + size_t(T) * H * 2);
     L.off_rs = o;    o = align256(o + size_t(T) * 4);
     L.off_h = o;     o = align256(o + P * I * 2);
-    L.off_ctrl = o;  o = align256(o + 16);
-    L.off_ccnt = o;  o = align256(o + size_t(T) * f.mt2 * 16 * 4);
+    L.off_ctrl = o;  o = align256(o + kLayerCtrl * 4);
     L.n_done = int(f.max_tiles1);
     L.off_done = o;  o = align256(o + size_t(L.n_done) * 4);
     L.n_cnt1 = int(f.max_tiles1 * f.mt1 * 16);
@@ -820,7 +823,6 @@ static cudaError_t launch_layer(const void* x, const float* logits, int T, int H
   p.x16 = reinterpret_cast<uint4*>(w + L.off_x16);
   p.rowscale = reinterpret_cast<float*>(w + L.off_rs);
   p.ctrl = reinterpret_cast<int*>(w + L.off_ctrl);
-  p.ccnt = reinterpret_cast<int*>(w + L.off_ccnt);
   p.tile_done = p.d.tile_done;
   p.cnt1 = p1.counters;
   p.cnt2 = p2.counters;
