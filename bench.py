@@ -160,7 +160,7 @@ def kernel_source_hash() -> str:
     counter taken on other code no longer describes the launches that run."""
     d = os.path.join(ROOT, "moe_expert_layer_renorm_b200", "csrc")
     h = hashlib.sha256()
-    for name in ("sm100.cuh", "ffn.cu", "decode.cu", "ffn_host.cu"):
+    for name in ("sm100.cuh", "ffn.cu", "decode.cu", "ffn_host.cu", "layer.cu"):
         with open(os.path.join(d, name), encoding="utf-8") as f:
             h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
