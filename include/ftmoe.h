@@ -423,14 +423,17 @@ FT_API int ft_gather_rows(const void* src, int n_src, int row_bytes, const int32
  * the pages' global LRU expert cache (FreeToken model guide, offload strategy,
  * OffloadMoeCache with per-(layer, expert) recency and a minimum-size guard;
  * sm89-moe-offload README, --moe-cache-size).  Each registered expert has a
- * pinned host copy of its slot image (layout->slot_bytes bytes); a miss is
- * filled by one cudaMemcpyAsync on the caller's copy stream, and the compute
- * stream waits on an event recorded after the copies.
+ * pinned host copy of its slot image (layout->slot_bytes bytes); the misses of
+ * one call are filled on the caller's copy stream, one cudaMemcpyAsync per run
+ * of consecutive slots whose host copies are consecutive too (register the
+ * banks of a layer in one page-locked block to get long runs), and the
+ * compute stream waits on an event recorded after the copies.
  * ------------------------------------------------------------------------- */
 typedef struct ft_slot_mgr ft_slot_mgr;
 
 typedef struct {
   int64_t hits, misses, evictions, bytes_h2d;
+  int64_t copies;   /* cudaMemcpyAsync calls the fills took (runs of consecutive slots and banks) */
 } ft_slot_stats_t;
 
 enum {

@@ -63,7 +63,8 @@ class Profile(ctypes.Structure):
 
 
 class SlotStats(ctypes.Structure):
-    _fields_ = [("hits", c_int64), ("misses", c_int64), ("evictions", c_int64), ("bytes_h2d", c_int64)]
+    _fields_ = [("hits", c_int64), ("misses", c_int64), ("evictions", c_int64), ("bytes_h2d", c_int64),
+                ("copies", c_int64)]
 
 
 _SIGS = {

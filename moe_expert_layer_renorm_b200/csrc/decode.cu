@@ -160,8 +160,14 @@ __device__ __forceinline__ void dec_stage(const uint8_t* st, int r_lo, int r_hi,
     const uint32_t wlo[4] = {clo.x, clo.y, clo.z, clo.w};
     const uint32_t whi[4] = {chi.x, chi.y, chi.z, chi.w};
     // the thread's 32 K span two 16-K scale blocks: words 0, 1 and words 2, 3
-    const uint32_t sl2[2] = {scale_pair_to_f16x2<FMT>(slo & 0xFFu, blo), scale_pair_to_f16x2<FMT>(slo >> 8, blo)};
-    const uint32_t sh2[2] = {scale_pair_to_f16x2<FMT>(shi & 0xFFu, bhi), scale_pair_to_f16x2<FMT>(shi >> 8, bhi)};
+    uint32_t sl2[2], sh2[2];
+    if (FMT == FT_SCALE_NVFP4) {   // both blocks' scales in one conversion, each then broadcast to a pair
+      e4m3x2_to_pairs(slo, sl2[0], sl2[1]);
+      e4m3x2_to_pairs(shi, sh2[0], sh2[1]);
+    } else {
+      sl2[0] = scale_pair_to_f16x2<FMT>(slo & 0xFFu, blo); sl2[1] = scale_pair_to_f16x2<FMT>(slo >> 8, blo);
+      sh2[0] = scale_pair_to_f16x2<FMT>(shi & 0xFFu, bhi); sh2[1] = scale_pair_to_f16x2<FMT>(shi >> 8, bhi);
+    }
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {   // word wd: 8 K = two MMA steps
       const int cb = (t & 1) * 4 + wd;   // the token values of those 8 K: 16-byte chunk of the box row

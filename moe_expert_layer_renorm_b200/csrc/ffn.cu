@@ -117,6 +117,17 @@ __device__ __forceinline__ uint32_t e8m0_pair_to_f16x2(uint32_t byte, int bias) 
 // the tensor's global (a power of two).
 __device__ __forceinline__ int mx_bias(float global) { return 127 + ilogbf(global); }
 
+// Two E4M3 scale bytes (the low byte is the first block's) -> (s0, s0) and
+// (s1, s1) in f16: one conversion and two byte permutes, about half the ALU
+// instructions of converting each byte on its own (the decode kernel's inner
+// loop is bound by the ALU pipe: measured 79.6 vs 82.0 us at decode_T64).
+__device__ __forceinline__ void e4m3x2_to_pairs(uint32_t two, uint32_t& p0, uint32_t& p1) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(uint16_t(two)));
+  p0 = __byte_perm(r, 0, 0x1010);
+  p1 = __byte_perm(r, 0, 0x3232);
+}
+
 // Scale byte of one 16-K block -> f16x2 (s, s) in the slot's format.
 template <int FMT>
 __device__ __forceinline__ uint32_t scale_pair_to_f16x2(uint32_t byte, int bias) {
@@ -147,9 +158,17 @@ template <int FMT>
 __device__ __forceinline__ void dequant_chunk(const uint4& c0, const uint4& c1, uint32_t sc, int bias,
                                               uint32_t (&o)[32]) {
   const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  uint32_t sp[4];
+  if (FMT == FT_SCALE_NVFP4) {
+    e4m3x2_to_pairs(sc & 0xFFFFu, sp[0], sp[1]);
+    e4m3x2_to_pairs(sc >> 16, sp[2], sp[3]);
+  } else {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) sp[b] = scale_pair_to_f16x2<FMT>((sc >> (8 * b)) & 0xFFu, bias);
+  }
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
-    const uint32_t s2 = scale_pair_to_f16x2<FMT>((sc >> (8 * b)) & 0xFFu, bias);
+    const uint32_t s2 = sp[b];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t q[4];

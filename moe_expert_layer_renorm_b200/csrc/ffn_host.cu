@@ -50,14 +50,18 @@ static int choose_splits(double units_est, int nkw, int num_sms, double split_co
 constexpr int kPreBN1 = 96, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 2, kPreDB1 = 2, kPreKC1 = 64;
 constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 3, kPreAS2 = 2, kPreDB2 = 2, kPreKC2 = 128;
 
-// Decode split-K: the smallest divisor of the K-stage count that gives every
-// SM a unit (a dynamic queue balances the rest, so waves do not matter).
+// Decode split-K: the largest divisor of the K-stage count that keeps the
+// units within one wave of the SMs (1 when there are more units than SMs).
+// At a few tokens the kernel is latency-bound: a second wave of units, and
+// each extra split's partial-sum exchange, lengthen the chain from the first
+// weight stage to the last output more than the idle SMs of one wave cost.
+// (Measured on a B200: decode_T1 33.7 vs 36.2 us per layer against the
+// smallest split count that fills every SM; wide_decode_T1 41.8 vs 45.3 us.)
 static int decode_splits(double units_est, int nkw, int num_sms, int* sps_out) {
   int best = 1;
   for (int s = 1; s <= std::min(nkw, 16); ++s) {
     if (nkw % s) continue;
-    best = s;
-    if (units_est * s >= num_sms) break;
+    if (units_est * s <= num_sms) best = s;
   }
   *sps_out = nkw / best;
   return best;

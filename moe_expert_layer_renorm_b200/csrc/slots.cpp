@@ -20,6 +20,7 @@
 // More distinct experts than capacity -> FT_ERR_CAPACITY (nothing changes).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <list>
@@ -179,13 +180,39 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
   std::vector<int32_t> table(table_len, -1);
   const size_t slot_bytes = size_t(m->layout.slot_bytes);
   std::vector<char> waited(ft_slot_mgr::kMarks, 0);   // one stream wait per distinct mark
-  for (int e : want) {
-    const uint64_t key = slot_key(layer, e);
-    auto it = m->resident.find(key);
-    if (it != m->resident.end()) {
-      table[e] = it->second.slot;
-      continue;
+  struct Fill {
+    int slot;
+    uint64_t key;
+    const uint8_t* src;
+    bool fail;   // an injected failure (test hook)
+  };
+  std::vector<Fill> fills;
+  // fills [from, end) did not happen: their slots are free again, their keys not resident
+  auto rollback = [&](size_t from) {
+    for (size_t r = from; r < fills.size(); ++r) {
+      auto it = m->resident.find(fills[r].key);
+      m->lru.erase(it->second.it);
+      m->resident.erase(it);
+      m->free_slots.push_back(fills[r].slot);
+      --m->stats.misses;
+      m->stats.bytes_h2d -= int64_t(slot_bytes);
     }
+    fills.resize(from);
+  };
+  // hits first; the misses then take their slots in the order of their host
+  // banks' addresses (stable: request order among equal addresses), so that
+  // consecutive slots receive consecutive banks and the copies coalesce
+  std::vector<int> misses;
+  for (int e : want) {
+    auto it = m->resident.find(slot_key(layer, e));
+    if (it != m->resident.end()) table[e] = it->second.slot;
+    else misses.push_back(e);
+  }
+  std::stable_sort(misses.begin(), misses.end(), [&](int a, int b) {
+    return m->banks[slot_key(layer, a)] < m->banks[slot_key(layer, b)];
+  });
+  for (int e : misses) {
+    const uint64_t key = slot_key(layer, e);
     int slot;
     if (!m->free_slots.empty()) {
       slot = m->free_slots.back();
@@ -196,6 +223,7 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
       for (auto r = m->lru.rbegin(); r != m->lru.rend(); ++r)
         if (!pinned.count(*r)) { victim = std::prev(r.base()); break; }
       if (victim == m->lru.end()) {
+        rollback(0);
         ftmoe::set_last_error("ft_slot_acquire: no evictable slot");
         return FT_ERR_CAPACITY;
       }
@@ -210,29 +238,50 @@ extern "C" int ft_slot_acquire(ft_slot_mgr* m, int layer, const int32_t* ids, in
     if (!m->host_only && mk >= 0 && !waited[mk]) {
       if (cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(copy), m->marks[mk], 0) != cudaSuccess) {
         m->free_slots.push_back(slot);
+        rollback(0);
         ftmoe::set_last_error("ft_slot_acquire: ordering the fill after compute failed");
         return FT_ERR_CUDA;
       }
       waited[mk] = 1;
     }
-    cudaError_t err = cudaSuccess;
+    bool fail = false;
     if (m->inject_failures > 0) {
       --m->inject_failures;
-      err = cudaErrorUnknown;
-    } else if (!m->host_only) {
-      err = cudaMemcpyAsync(m->pool + size_t(slot) * slot_bytes, m->banks[key], slot_bytes,
-                            cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(copy));
+      fail = true;
     }
-    if (err != cudaSuccess) {
-      m->free_slots.push_back(slot);   // the slot holds nothing valid now
-      ftmoe::set_last_error("ft_slot_acquire: host-to-device fill failed");
-      return FT_ERR_CUDA;
-    }
+    fills.push_back(Fill{slot, key, static_cast<const uint8_t*>(m->banks[key]), fail});
     m->lru.push_front(key);
     m->resident[key] = ft_slot_mgr::Entry{slot, m->lru.begin()};
     table[e] = slot;
     ++m->stats.misses;
     m->stats.bytes_h2d += int64_t(slot_bytes);
+  }
+  // The fills, one cudaMemcpyAsync per run of consecutive slots whose host
+  // banks are consecutive too (banks registered in one page-locked block, and
+  // slots freed in the order they were handed out, make long runs): each copy
+  // has a fixed cost on the copy engine, so 128 fills of one layer become a
+  // few large copies.  Every wait above is already enqueued before them.  A
+  // failed copy leaves its run and every later one not resident.
+  std::sort(fills.begin(), fills.end(), [](const Fill& a, const Fill& b) { return a.slot < b.slot; });
+  for (size_t i = 0; i < fills.size();) {
+    size_t j = i + 1;
+    bool fail = fills[i].fail;
+    while (j < fills.size() && fills[j].slot == fills[j - 1].slot + 1 &&
+           fills[j].src == fills[j - 1].src + slot_bytes) {
+      fail = fail || fills[j].fail;
+      ++j;
+    }
+    cudaError_t err = fail ? cudaErrorUnknown : cudaSuccess;
+    if (!fail && !m->host_only)
+      err = cudaMemcpyAsync(m->pool + size_t(fills[i].slot) * slot_bytes, fills[i].src, (j - i) * slot_bytes,
+                            cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(copy));
+    if (err != cudaSuccess) {
+      rollback(i);   // this run and the later ones hold nothing valid
+      ftmoe::set_last_error("ft_slot_acquire: host-to-device fill failed");
+      return FT_ERR_CUDA;
+    }
+    ++m->stats.copies;
+    i = j;
   }
   m->host_table = table;
   for (int e : want) m->prev_slots.push_back(table[e]);

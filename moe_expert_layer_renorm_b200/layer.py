@@ -220,7 +220,8 @@ class SlotManager:
     def stats(self) -> dict:
         s = _lib.SlotStats()
         _lib.check(_lib.lib().ft_slot_stats(self.h, ctypes.byref(s)))
-        return {"hits": s.hits, "misses": s.misses, "evictions": s.evictions, "bytes_h2d": s.bytes_h2d}
+        return {"hits": s.hits, "misses": s.misses, "evictions": s.evictions, "bytes_h2d": s.bytes_h2d,
+                "copies": s.copies}
 
     def close(self) -> None:
         if self.h:

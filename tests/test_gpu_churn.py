@@ -50,3 +50,36 @@ def test_churn_routes_to_hot_sets():
         lg = churn.step_logits(cfg, hs, 1, d, 5)
         top = np.argsort(-lg, axis=1)[:, :cfg.k]
         assert set(top.ravel().tolist()) <= set(hs[1, d].tolist())
+
+
+@pytest.mark.gpu
+def test_prefill_streaming_matches_resident(cuda_device):
+    # the prefill streaming order: 3 layers of 512 tokens, every expert of a
+    # layer used (k = 4 of E = 16, one domain), a pool of two layers' worth,
+    # so each layer's 16 experts are filled from the host while the previous
+    # layer runs, evicting the slots of the layer before it; the groups (~128
+    # rows per expert) take the tcgen05 kernels.  Outputs are bit-identical to
+    # the same layers with every expert resident, and the fills coalesce.
+    cfg = churn.ChurnConfig(T=512, E=16, k=4, H=256, I=256, layers=3, domains=1, hot=16, capacity=32)
+    hs = churn.hot_sets(cfg)
+    banks = churn.ExpertBanks(cfg, hs, keep_device=True)
+    run = churn.ChurnRun(cfg, banks)
+    outs, all_logits = [], []
+    for step in range(3):
+        logits = [torch.from_numpy(churn.step_logits(cfg, hs, l, 0, step)).cuda() for l in range(cfg.layers)]
+        all_logits.append(logits)
+        run.step(logits, "prefetch", outs)
+    torch.cuda.synchronize()
+    st = run.mgr.stats()
+    assert st["misses"] == 16 * 3 * 3 and st["evictions"] > 0
+    assert st["copies"] < st["misses"]          # runs of consecutive slots and banks
+    ref = MoELayer(cfg.T, cfg.E, cfg.k, cfg.H, cfg.I)
+    i = 0
+    for logits in all_logits:
+        for l in range(cfg.layers):
+            y = ref.forward(run.x[l], logits[l], banks.resident_table(cfg, l), banks.resident)
+            torch.cuda.synchronize()
+            assert torch.equal(y, outs[i]), f"layer {l}, output {i}"
+            assert torch.isfinite(y).all()
+            i += 1
+    run.mgr.close()

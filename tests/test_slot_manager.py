@@ -143,3 +143,24 @@ def test_layers_are_separate_keys():
     b = _acquire(m, 1, [7])
     assert a[7] != b[7]
     assert m.stats()["misses"] == 2
+
+
+def test_fills_coalesce_into_runs_of_consecutive_slots_and_banks():
+    # banks of one layer in one block: the misses of a call become one copy per run of
+    # consecutive slots whose banks are consecutive too, whatever the request order
+    cap, E = 8, 16
+    lay = _lib.slot_layout(256, 512, cap)
+    m = SlotManager(cap, lay, host_only=True)
+    nbytes = int(lay.slot_bytes)
+    block = (ctypes.c_uint8 * (nbytes * E))()
+    base = ctypes.addressof(block)
+    for e in range(E):
+        m.register_host(0, e, base + e * nbytes)
+    t = _acquire(m, 0, [3, 0, 2, 1])            # four free slots, banks 0..3: one run
+    st = m.stats()
+    assert st["misses"] == 4 and st["copies"] == 1
+    assert [t[e] for e in range(4)] == [0, 1, 2, 3]   # slots follow the banks' order
+    t = _acquire(m, 0, [9, 5])                   # banks 5 and 9 are not adjacent: two copies
+    st2 = m.stats()
+    assert st2["misses"] == 6 and st2["copies"] == 3
+    assert sorted([t[5], t[9]]) == [4, 5]
