@@ -71,7 +71,11 @@ struct FfnParams {
 // KC: K per chunk (64 or 128), the unit of one dequantised A slot, one
 // token stage and one operand hand-over to the MMA warp.  A chunk of 128
 // halves the per-chunk costs (barriers, hand-over, commits) per MMA.
-template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC>
+// AM: where the dequantised A operand lives -- 0: tensor memory (the MMA's TS
+// form, tcgen05.st from the dequantising warps), 1: shared memory (SS form,
+// 128-byte-swizzled K-major rows like the token boxes), which leaves tensor
+// memory to the accumulators.
+template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC, int AM = 0>
 struct FfnCfg {
   static constexpr int kAtoms = KC / kAtomK;                 // swizzle atoms (token boxes) per chunk
   static constexpr int kCPW = kKW / KC;                      // chunks per weight stage
@@ -80,10 +84,12 @@ struct FfnCfg {
   static constexpr int kBAtomBytes = BN * 128;
   static constexpr int kBStageBytes = kAtoms * kBAtomBytes;
   static constexpr int kBBytes = BS * kBStageBytes;
+  static constexpr int kAAtomBytes = 128 * 128;               // one 64-K atom of 128 weight rows, f16
+  static constexpr int kABytes = AM ? AS * NMAT * kAtoms * kAAtomBytes : 0;
   static constexpr int kNumBars = 2 * WS + 2 * BS + 2 * AS + 2 * DB + 1;
-  static constexpr int kSmemBytes = 1024 /*align slack*/ + kWBytes + kBBytes + BN * 4 + kNumBars * 8 + 64;
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kWBytes + kBBytes + kABytes + BN * 4 + kNumBars * 8 + 64;
   static constexpr int kDCols = DB * NMAT * BN;
-  static constexpr int kTmemCols = kDCols + AS * NMAT * kACols;
+  static constexpr int kTmemCols = kDCols + (AM ? 0 : AS * NMAT * kACols);
   static_assert(KC == 64 || KC == 128, "chunk size");
   static_assert(kTmemCols <= 512, "tensor memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
@@ -258,19 +264,20 @@ __device__ __forceinline__ float token_factor(const FfnParams& p, int row) {
   return p.rowscale != nullptr ? __ldg(p.rowscale + row) : 1.0f;
 }
 
-template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC, int FMT>
+template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC, int FMT, int AM>
 __global__ void __launch_bounds__(kThreads, 1)
 ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0,
                 const __grid_constant__ CUtensorMap tm_scales0, const __grid_constant__ CUtensorMap tm_codes1,
                 const __grid_constant__ CUtensorMap tm_scales1, const __grid_constant__ CUtensorMap tm_act) {
   pdl_wait();   // dependents are triggered at the end (see below)
-  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB, KC>;
+  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB, KC, AM>;
   constexpr int kCPW = Cfg::kCPW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* w_smem = smem;
   uint8_t* b_smem = smem + Cfg::kWBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + Cfg::kBBytes);
+  uint8_t* a_smem = b_smem + Cfg::kBBytes;   // AM = 1: AS x NMAT x kAtoms atoms of 16 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(a_smem + Cfg::kABytes);
   uint64_t* w_full = bars;
   uint64_t* w_empty = w_full + WS;
   uint64_t* b_full = w_empty + WS;
@@ -372,16 +379,28 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
           const int as = q % AS, bs = q % BS;
           const uint64_t bd = make_sdesc_sw128(smem_u32(b_smem + bs * Cfg::kBStageBytes));
           const uint32_t d0 = tmem + ds * NMAT * BN;
-          const uint32_t a0 = tmem + Cfg::kDCols + as * NMAT * Cfg::kACols;
           const uint32_t acc0 = c > kc0 ? 1u : 0u;
+          if (AM) {   // A: atom (as, m, j / 4) of shared memory, +32 bytes per K slice in it
+            const uint64_t ad = make_sdesc_sw128(smem_u32(a_smem + as * NMAT * Cfg::kAtoms * Cfg::kAAtomBytes));
 #pragma unroll
-          for (int m = 0; m < NMAT; ++m) mma_ts_f16(d0 + m * BN, a0 + m * Cfg::kACols, bd, idesc, acc0);
+            for (int j = 0; j < KC / 16; ++j)
 #pragma unroll
-          for (int j = 1; j < KC / 16; ++j)
+              for (int m = 0; m < NMAT; ++m)
+                mma_ss_f16(d0 + m * BN,
+                           ad + uint64_t(((m * Cfg::kAtoms + j / 4) * Cfg::kAAtomBytes >> 4) + 2 * (j % 4)),
+                           bd + uint64_t((j / 4) * (Cfg::kBAtomBytes >> 4) + 2 * (j % 4)), idesc,
+                           j > 0 ? 1u : acc0);
+          } else {
+            const uint32_t a0 = tmem + Cfg::kDCols + as * NMAT * Cfg::kACols;
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m)   // K slice j: atom j / 4 (+kBAtomBytes), +32 bytes per slice in it
-              mma_ts_f16_acc(d0 + m * BN, a0 + m * Cfg::kACols + 8 * j,
-                             bd + uint64_t((j / 4) * (Cfg::kBAtomBytes >> 4) + 2 * (j % 4)), idesc);
+            for (int m = 0; m < NMAT; ++m) mma_ts_f16(d0 + m * BN, a0 + m * Cfg::kACols, bd, idesc, acc0);
+#pragma unroll
+            for (int j = 1; j < KC / 16; ++j)
+#pragma unroll
+              for (int m = 0; m < NMAT; ++m)   // K slice j: atom j / 4 (+kBAtomBytes), +32 bytes per slice in it
+                mma_ts_f16_acc(d0 + m * BN, a0 + m * Cfg::kACols + 8 * j,
+                               bd + uint64_t((j / 4) * (Cfg::kBAtomBytes >> 4) + 2 * (j % 4)), idesc);
+          }
           mma_commit(&a_empty[as]);
           mma_commit(&b_empty[bs]);
         }
@@ -492,11 +511,23 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
               const uint32_t sc = *reinterpret_cast<const uint32_t*>(base + kCodesBytes + row * 16 + t * 4);
               uint32_t o[32];
               dequant_chunk<FMT>(c0, c1, sc, bias[m], o);
-              tmem_st_32x32b_x32(tmem + lane_base + Cfg::kDCols + (as * NMAT + m) * Cfg::kACols + h * 32, o);
+              if (AM) {   // row `row` of the atom, its eight 16-byte chunks 128-byte swizzled
+                uint8_t* arow = a_smem + ((as * NMAT + m) * Cfg::kAtoms + h) * Cfg::kAAtomBytes + row * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  *reinterpret_cast<uint4*>(arow + ((j ^ (row & 7)) << 4)) =
+                      make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+              } else {
+                tmem_st_32x32b_x32(tmem + lane_base + Cfg::kDCols + (as * NMAT + m) * Cfg::kACols + h * 32, o);
+              }
             }
           }
-          tmem_wait_st();
-          tc_fence_before();
+          if (AM) {
+            fence_proxy_async_smem();   // the generic stores, visible to the MMA's operand reads
+          } else {
+            tmem_wait_st();
+            tc_fence_before();
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[as]);
         }

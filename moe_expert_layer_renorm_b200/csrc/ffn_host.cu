@@ -13,6 +13,7 @@ struct GemmShape { int bn, splits, sps, ws, bs, as, db; };
 
 struct FfnPlan {
   bool decode;
+  bool gu_smem;        // gate/up GEMM in the large-group shape (A in shared memory)
   GemmShape g1, g2;
   int mt1, mt2, nkw1, nkw2, nkc1, nkc2;
   long long max_tiles1, max_tiles2;
@@ -44,11 +45,21 @@ static int choose_splits(double units_est, int nkw, int num_sms, double split_co
 }
 
 // Prefill tile shapes <token rows (MMA N), weight stages, token stages, A
-// stages, accumulator buffers, K per chunk> of the two tcgen05 GEMMs.
-// Tensor memory holds DB * NMAT * BN accumulator columns plus
-// AS * NMAT * KC / 2 for A.
-constexpr int kPreBN1 = 96, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 2, kPreDB1 = 2, kPreKC1 = 64;
-constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 3, kPreAS2 = 2, kPreDB2 = 2, kPreKC2 = 128;
+// stages, accumulator buffers, K per chunk, A in shared memory> of the two
+// tcgen05 GEMMs.  Tensor memory holds DB * NMAT * BN accumulator columns plus,
+// with A in tensor memory, AS * NMAT * KC / 2 for A.
+//   gate/up, groups of up to a few hundred rows: A in tensor memory, 96-row
+//     token tiles (the deeper weight ring keeps the weight stream going);
+//   gate/up, large groups (mean >= kGateUpSmemRows rows per active expert):
+//     A in shared memory, so that tensor memory holds two 128-column
+//     accumulator buffers per matrix, with three A slots (measured on a B200:
+//     wide_T8192 gate/up 1213 vs 1392 us, prefill_zipf_T4096 314 vs 330 us;
+//     slots512_T8192 with 160 rows per expert 581 vs 525 us, so it keeps the
+//     first shape).
+constexpr int kPreBN1 = 96, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 2, kPreDB1 = 2, kPreKC1 = 64, kPreAM1 = 0;
+constexpr int kPreBN1S = 128, kPreWS1S = 2, kPreBS1S = 3, kPreAS1S = 3, kPreDB1S = 2, kPreKC1S = 64, kPreAM1S = 1;
+constexpr double kGateUpSmemRows = 192.0;
+constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 3, kPreAS2 = 2, kPreDB2 = 2, kPreKC2 = 128, kPreAM2 = 0;
 
 // Decode split-K: the largest divisor of the K-stage count that keeps the
 // units within one wave of the SMs (1 when there are more units than SMs).
@@ -90,7 +101,9 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
     pl.g1 = {kDecBN, 1, 0, 4, 0, 0, 0};
     pl.g2 = {kDecBN, 1, 0, 4, 0, 0, 0};
   } else {
-    pl.g1 = {kPreBN1, 1, 0, kPreWS1, kPreBS1, kPreAS1, kPreDB1};
+    pl.gu_smem = mean_rows >= kGateUpSmemRows;
+    pl.g1 = pl.gu_smem ? GemmShape{kPreBN1S, 1, 0, kPreWS1S, kPreBS1S, kPreAS1S, kPreDB1S}
+                       : GemmShape{kPreBN1, 1, 0, kPreWS1, kPreBS1, kPreAS1, kPreDB1};
     pl.g2 = {kPreBN2, 1, 0, kPreWS2, kPreBS2, kPreAS2, kPreDB2};
   }
   const double tiles_per_expert1 = std::max(1.0, ceil(mean_rows / pl.g1.bn));
@@ -216,13 +229,13 @@ static bool make_act_map(const void* base, int rows, int K, int box_rows, CUtens
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC, int FMT>
+template <int NMAT, int BN, int WS, int BS, int AS, int DB, int KC, int FMT, int AM>
 static cudaError_t launch_gemm(const FfnParams& p, int grid, const CUtensorMap& c0, const CUtensorMap& s0,
                                const CUtensorMap& c1, const CUtensorMap& s1, const CUtensorMap& act,
                                cudaStream_t s) {
   ProfileScope prof(NMAT == 2 ? FT_KERNEL_GEMM_GATE_UP : FT_KERNEL_GEMM_DOWN, s);
-  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB, KC>;
-  auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB, KC, FMT>;
+  using Cfg = FfnCfg<NMAT, BN, WS, BS, AS, DB, KC, AM>;
+  auto kern = ffn_gemm_kernel<NMAT, BN, WS, BS, AS, DB, KC, FMT, AM>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
@@ -293,7 +306,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
   if (err != cudaSuccess) return err;
 
   CUtensorMap tm_x, tm_h;
-  if (!make_act_map(x16, T * k, H, pl.decode ? kDecBN : kPreBN1, &tm_x) ||
+  if (!make_act_map(x16, T * k, H, pl.decode ? kDecBN : pl.g1.bn, &tm_x) ||
       !make_act_map(h, T * k, I, pl.decode ? kDecBN : kPreBN2, &tm_h)) {
     *why = "cuTensorMapEncodeTiled failed for the activations";
     return cudaErrorInvalidValue;
@@ -350,14 +363,17 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
     const int grid = int(std::min<long long>(num_sms, pl.max_units1 + pl.max_units2));
     err = L.scale_format == FT_SCALE_MXFP4 ? launch_decode<FT_SCALE_MXFP4>(dp, grid, tmc, tms, tm_x, tm_h, s)
                                            : launch_decode<FT_SCALE_NVFP4>(dp, grid, tmc, tms, tm_x, tm_h, s);
-  } else if (L.scale_format == FT_SCALE_MXFP4) {
-    err = launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1, FT_SCALE_MXFP4>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
-    if (err == cudaSuccess)
-      err = launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2, FT_SCALE_MXFP4>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   } else {
-    err = launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1, FT_SCALE_NVFP4>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    const bool mx = L.scale_format == FT_SCALE_MXFP4;
+    if (pl.gu_smem)
+      err = mx ? launch_gemm<2, kPreBN1S, kPreWS1S, kPreBS1S, kPreAS1S, kPreDB1S, kPreKC1S, FT_SCALE_MXFP4, kPreAM1S>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s)
+               : launch_gemm<2, kPreBN1S, kPreWS1S, kPreBS1S, kPreAS1S, kPreDB1S, kPreKC1S, FT_SCALE_NVFP4, kPreAM1S>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    else
+      err = mx ? launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1, FT_SCALE_MXFP4, kPreAM1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s)
+               : launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1, FT_SCALE_NVFP4, kPreAM1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
     if (err == cudaSuccess)
-      err = launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2, FT_SCALE_NVFP4>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
+      err = mx ? launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2, FT_SCALE_MXFP4, kPreAM2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s)
+               : launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2, FT_SCALE_NVFP4, kPreAM2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   }
   return err;
 }

@@ -28,9 +28,11 @@ def test_layer_full_parity(cuda_device, name):
     G.check_output(run, w.k)
 
 
-@pytest.mark.parametrize("H,I,E,k,T", [(320, 448, 8, 2, 40), (256, 256, 4, 4, 100), (576, 320, 16, 3, 333)])
+@pytest.mark.parametrize("H,I,E,k,T", [(320, 448, 8, 2, 40), (256, 256, 4, 4, 100), (576, 320, 16, 3, 333),
+                                         (320, 448, 4, 2, 600), (576, 2880, 3, 2, 700)])
 def test_ragged_shapes(cuda_device, H, I, E, k, T):
-    # K not a multiple of 256, output features not a multiple of 128, groups spanning several tiles
+    # K not a multiple of 256, output features not a multiple of 128, groups spanning several tiles; the
+    # last two have hundreds of rows per expert (the gate/up GEMM's large-group shape)
     w = inputs.custom_workload(W["tiny"], H=H, I=I, E=E, k=k, T=T, seed=4242 + H)
     run = G.run_gpu(w)
     G.check_routing(run, w.k)

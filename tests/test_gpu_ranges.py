@@ -21,10 +21,12 @@ from tests import gpu_helpers as G
 pytestmark = pytest.mark.gpu
 W = inputs.WORKLOADS
 
-# decode kernel: a few rows per expert; prefill (tcgen05) kernel: 100 rows per expert
+# decode kernel: a few rows per expert; prefill (tcgen05) kernels: 100 rows per expert, and 400 (the
+# gate/up GEMM's large-group shape, A in shared memory)
 SHAPES = {
     "decode": inputs.custom_workload(W["tiny"], T=40, seed=5151),
     "prefill": inputs.custom_workload(W["tiny"], H=256, I=256, E=4, k=4, T=100, seed=5152),
+    "prefill_large": inputs.custom_workload(W["tiny"], H=256, I=256, E=4, k=4, T=400, seed=5153),
 }
 
 

@@ -64,3 +64,14 @@ def test_mxfp4_prefill_layer_parity_sampled(cuda_device):
     pool, st = G.build_pool(w, fmt=_lib.FT_SCALE_MXFP4)
     run = G.run_gpu(w, pool=pool, slot_table=st)
     G.check_output(run, w.k, tokens=np.arange(0, 1024, 37))
+
+
+def test_mxfp4_large_groups_layer_parity(cuda_device):
+    # 600 tokens over 4 experts at top-2 (~300 rows per expert): the gate/up GEMM's large-group shape
+    # (A operand in shared memory), with the MXFP4 scale decode, K = 320 (not a multiple of 256)
+    w = inputs.custom_workload(W["tiny"], H=320, I=448, E=4, k=2, T=600, seed=6161)
+    pool, st = G.build_pool(w, fmt=_lib.FT_SCALE_MXFP4)
+    run = G.run_gpu(w, pool=pool, slot_table=st)
+    G.check_routing(run, w.k)
+    G.check_output(run, w.k)
+
