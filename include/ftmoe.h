@@ -155,6 +155,12 @@ FT_API int ft_pack_slot(const float* w, int mat, const ft_nvfp4_slot_layout* lay
  *   topk_ids  device int32 [T, k]  (out)
  *   topk_w    device fp32  [T, k]  (out)
  * Requires 1 <= k <= min(E, 32), E <= 1024.
+ * Pages: the routers of the MoE families in "FreeToken model guide" (its
+ * model table: Qwen3.6-35B-A3B, gpt-oss, Gemma-4 A4B and the like) and the
+ * "MoE serving" of the About page's "Fast Edge-Native Runtime" select k
+ * experts per token; no page writes the router down, so the two weightings
+ * (softmax over all experts then renormalised over the k, or softmax over
+ * the k) are this library's reading of a top-k router.
  */
 FT_API int ft_moe_route(const float* logits, int T, int E, int k, int mode,
                  int32_t* topk_ids, float* topk_w, ft_stream_t stream);
@@ -168,6 +174,12 @@ FT_API int ft_moe_route(const float* logits, int T, int E, int k, int mode,
  *   ws              device workspace of ft_moe_permute_workspace_size bytes
  * Deterministic (no atomics decide any order).  Ids outside [0, E) set
  * FT_DEV_BAD_INDEX.
+ * Pages: the grouping of tokens per expert that a grouped expert GEMM needs
+ * (the "sm89-moe-offload" fork README, "Key customizations": the NVFP4
+ * prefill MoE kernel for M >= 2048 rows) is not described on any page; a
+ * stable counting sort by expert is the plainest reading.  Determinism
+ * follows the About page's "graph-compatible execution" ("Fast Edge-Native
+ * Runtime"): the same inputs replay to the same bytes.
  */
 FT_API int ft_moe_permute(const int32_t* topk_ids, int T, int k, int E,
                    int32_t* expert_offsets, int32_t* perm_src, int32_t* pair_to_row,
@@ -244,6 +256,14 @@ FT_API int ft_moe_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
  *   ws             device workspace of ft_moe_ffn_workspace_size bytes, 256-B aligned
  * A non-empty group whose slot is -1 sets FT_DEV_NOT_RESIDENT and its rows are
  * left unwritten.  H and I must be multiples of 64 and match the layout.
+ * Pages: NVFP4 expert weights and their MoE kernels ("FreeToken model
+ * guide", the NVFP4 releases of each family and --quant-backend
+ * moe.nvfp4=marlin|b12x|triton; the "sm89-moe-offload" fork README,
+ * "Production configuration" and "Key customizations": the wide-load NVFP4
+ * prefill MoE kernel, prior art for sm_89); experts addressed through the
+ * expert cache (About page, "Fast Edge-Native Runtime": global LRU expert
+ * caching).  The SwiGLU expert (silu(gate) * up, then down) is the expert
+ * of the MoE families the model guide lists; no page writes it down.
  */
 FT_API int ft_moe_ffn_nvfp4(const void* x, int T, int H, int I, int E, int k,
                      const int32_t* perm_src, const int32_t* expert_offsets,
@@ -258,6 +278,10 @@ FT_API size_t ft_moe_ffn_workspace_size(int T, int H, int I, int E, int k);
  *   out_perm device fp32 [T*k, H], pair_to_row device int32 [T*k],
  *   topk_w device fp32 [T, k], y device fp32 [T, H] (out).  H % 4 == 0;
  *   out_perm and y 16-byte aligned.
+ * Pages: the weighted return of each token's k expert outputs is the last
+ * step of the "MoE serving" of the About page ("Fast Edge-Native Runtime");
+ * no page writes it down, and the fixed summation order is this library's
+ * reading of its "graph-compatible execution" (replays give the same bytes).
  */
 FT_API int ft_moe_combine(const void* out_perm, const int32_t* pair_to_row, const float* topk_w,
                    int T, int k, int H, void* y, ft_stream_t stream);
@@ -309,6 +333,13 @@ FT_API size_t ft_moe_layer_workspace_size(int T, int H, int I, int E, int k);
  *   global_scale device fp32 [1]             (out)
  *   ws           device workspace, >= 4 bytes (holds amax)
  * The destinations may point inside a slot (see ft_nvfp4_slot_layout).
+ * Pages: NVFP4 is the expert format of the served checkpoints ("FreeToken
+ * model guide", the -NVFP4 releases and --quant-backend moe.nvfp4; the
+ * "sm89-moe-offload" fork README, "Production configuration"; About page,
+ * "Broad MoE & Ecosystem Support": MXFP4, NVFP4, FP8, BF16).  No page defines
+ * the format's bits; the layout above is NVIDIA's published NVFP4 (E2M1
+ * values, one E4M3 scale per 16, an fp32 tensor scale), and the choice of g
+ * (amax / (6 * 448)) is this library's reading.
  */
 FT_API int ft_nvfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* scales, int ld_scale,
                   float* global_scale, void* ws, ft_stream_t stream);
@@ -316,7 +347,7 @@ FT_API int ft_nvfp4_pack(const float* w, int N, int K, uint8_t* codes, uint8_t* 
 /*
  * MXFP4 pack of one fp32 tensor [N, K] (K % 32 == 0): the OCP Microscaling
  * (MX) conversion, which the pages name as an expert format beside NVFP4
- * ("FlashML-org / FreeToken" about page, quantization formats) without
+ * ("FlashML-org / FreeToken" About page, "Broad MoE & Ecosystem Support") without
  * defining it.  Per 32-block b of a row:
  *   x_b = floor(log2 amax_b) - 2, clamped to [-127, 127]; -127 if amax_b = 0
  *   scale byte s_b = x_b + 127, written at scales[row][2b] and [2b + 1]
