@@ -4,10 +4,14 @@
 //   1. per-chunk histograms of the expert ids            (one CTA per chunk)
 //   2. expert offsets = exclusive scan of the totals, and
 //      base[c][e] = offsets[e] + sum_{c' < c} count[c'][e] (one CTA)
-//   3. scatter: one warp walks its chunk 32 pairs at a time; pairs of the same
-//      expert inside a step are ranked with __match_any_sync, so a pair's row
-//      is base + (number of earlier pairs of its expert).  No atomic decides
-//      any order, so the result is deterministic.
+//   3. scatter: the CTA stages its chunk's ids in shared memory and cuts the
+//      chunk into one run of consecutive pairs per warp; per-warp counts give
+//      each warp its first row per expert (the chunk's base plus the counts
+//      of the warps before it).  Each warp then walks its run 32 pairs at a
+//      time; pairs of the same expert inside a step are ranked with
+//      __match_any_sync, so a pair's row is its warp's base + (number of
+//      earlier pairs of its expert).  No atomic decides any order, so the
+//      result is deterministic.
 // Small inputs (one chunk) run all three steps in a single CTA.
 #include "sm100.cuh"
 
@@ -15,6 +19,7 @@ namespace ftmoe {
 
 constexpr int kPermChunk = 1024;
 constexpr int kMaxExperts = 1024;
+constexpr int kScatterThreads = 256;
 
 __device__ __forceinline__ bool valid_expert(int e, int E) { return e >= 0 && e < E; }
 
@@ -122,35 +127,65 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
   pdl_enter();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
+  constexpr int kBatch = 8;   // loads in flight per thread
   int total = 0;
   if (e < E)
-    for (int c = 0; c < nchunks; ++c) total += counts[size_t(c) * E + e];
+    for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
+      int n[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) n[i] = c0 + i < nchunks ? counts[size_t(c0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) total += n[i];
+    }
   const int ex = block_exclusive_scan(total, warp_sums);
   if (e < E) {
     offsets[e] = ex;
     int run = ex;
-    for (int c = 0; c < nchunks; ++c) {  // counts become per-chunk base rows
-      const int n = counts[size_t(c) * E + e];
-      counts[size_t(c) * E + e] = run;
-      run += n;
+    for (int c0 = 0; c0 < nchunks; c0 += kBatch) {  // counts become per-chunk base rows
+      int n[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) n[i] = c0 + i < nchunks ? counts[size_t(c0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        if (c0 + i < nchunks) {
+          counts[size_t(c0 + i) * E + e] = run;
+          run += n[i];
+        }
     }
   }
   if (e == E - 1) offsets[E] = ex + total;
 }
 
-__global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __restrict__ ids, int P, int E,
+__global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(const int32_t* __restrict__ ids, int P, int E,
                                                               const int32_t* __restrict__ bases,
                                                               int32_t* __restrict__ perm_src,
                                                               int32_t* __restrict__ pair_to_row) {
   pdl_enter();
-  __shared__ int cursor[kMaxExperts];
-  const int c = blockIdx.x;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] = bases[size_t(c) * E + e];
+  constexpr int kWarps = kScatterThreads / 32, kRun = kPermChunk / kWarps;
+  __shared__ int32_t sids[kPermChunk];
+  __shared__ int cursor[kWarps][kMaxExperts];   // per warp: its count, then its first row, per expert
+  const int c = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cursor[i / E][i % E] = 0;
+  for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) sids[p - p0] = __ldg(ids + p);
   __syncthreads();
-  if (threadIdx.x < 32) {
-    const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
-    scatter_chunk_warp<false>(ids, p0, p1, E, cursor, perm_src, pair_to_row, P);
+  const int q0 = min(p1, p0 + warp * kRun), q1 = min(p1, q0 + kRun);   // this warp's run
+  for (int p = q0 + lane; p < q1; p += 32) {
+    const int e = sids[p - p0];
+    if (valid_expert(e, E)) atomicAdd(&cursor[warp][e], 1);
   }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = bases[size_t(c) * E + e];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int n = cursor[w][e];
+      cursor[w][e] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  if (q0 < q1) scatter_chunk_warp<true>(sids + (q0 - p0), q0, q1, E, cursor[warp], perm_src, pair_to_row, P);
 }
 
 // Route and permute in one CTA for small batches (T <= kFusedMaxT tokens,
@@ -241,7 +276,7 @@ static cudaError_t launch_permute(const int32_t* ids, int T, int k, int E, int32
   }
   if (e != cudaSuccess) return e;
   ProfileScope prof(FT_KERNEL_PERMUTE, s);
-  return launch_pdl(permute_scatter_kernel, dim3(nchunks), dim3(256), 0, s, ids, P, E,
+  return launch_pdl(permute_scatter_kernel, dim3(nchunks), dim3(kScatterThreads), 0, s, ids, P, E,
                     static_cast<const int32_t*>(counts), perm_src, pair_to_row);
 }
 

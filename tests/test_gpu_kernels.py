@@ -76,6 +76,29 @@ def test_permute_bit_exact(cuda_device, T, E, k):
         assert np.array_equal(b.cpu().numpy(), p2r)
 
 
+def test_permute_bad_id_in_a_large_batch_sets_status(cuda_device):
+    # several chunks: the out-of-range id sits in the second chunk, in a warp's run
+    # that is not the first; the bad pair gets no row and the call records the status
+    g = np.random.default_rng(77)
+    T, k, E = 2000, 2, 16
+    ids = np.stack([g.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    ids[700, 1] = 99
+    d_ids = torch.from_numpy(ids).cuda()
+    P = T * k
+    o = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    a = torch.full((P,), -7, dtype=torch.int32, device="cuda")
+    b = torch.full((P,), -7, dtype=torch.int32, device="cuda")
+    wsb = _lib.permute_workspace_size(T, k, E)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+    _lib.device_status(clear=True)
+    _lib.permute(d_ids.data_ptr(), T, k, E, o.data_ptr(), a.data_ptr(), b.data_ptr(), ws.data_ptr(), wsb,
+                 _stream())
+    torch.cuda.synchronize()
+    assert _lib.device_status(clear=True) == _lib.FT_DEV_BAD_INDEX
+    assert int(b.cpu().numpy()[700 * k + 1]) == -7
+    assert int(o.cpu().numpy()[E]) == P - 1
+
+
 def test_permute_bad_id_sets_status(cuda_device):
     _lib.device_status(clear=True)
     ids = torch.tensor([[0, 9]], dtype=torch.int32, device="cuda")
