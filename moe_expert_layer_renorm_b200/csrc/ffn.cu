@@ -830,11 +830,11 @@ __device__ __forceinline__ int prep_row_exp(float m) {
 // exactly down to 2^-17); smaller elements round, to f16 subnormals, with an
 // absolute error of at most 2^-25 in converted units, below 2^-38 max|x[t]|.
 // Rows in permuted order make each expert group's tokens one contiguous
-// block, so the GEMM loads them as plain tiles.  Rows of up to 3072 values
-// are read once into registers with all loads in flight together (the
+// block, so the GEMM loads them as plain tiles.  Rows of up to 256 * kRegVec
+// values are read once into registers with all loads in flight together (the
 // kernel is latency-bound at decode sizes); longer rows are read twice.
+template <int kRegVec>   // 16-byte vectors per lane kept in registers
 __device__ void prep_rows(const PrepParams& p, int b) {
-  constexpr int kRegVec = 12;                    // 16-byte vectors per lane kept in registers
   const int lane = threadIdx.x & 31;
   const int r = b * (blockDim.x / 32) + threadIdx.x / 32;
   if (r >= p.P) return;
@@ -842,8 +842,8 @@ __device__ void prep_rows(const PrepParams& p, int b) {
   const int nv = p.H / 8;
   const uint4* row = p.x + size_t(t) * nv;
   uint4* out = p.x_perm + size_t(r) * nv;
-  if (nv <= 32 * kRegVec) {
-    uint4 v[kRegVec];
+  if (kRegVec > 0 && nv <= 32 * kRegVec) {
+    uint4 v[kRegVec > 0 ? kRegVec : 1];
 #pragma unroll
     for (int i = 0; i < kRegVec; ++i) {
       const int c = lane + 32 * i;
@@ -877,10 +877,15 @@ __device__ void prep_rows(const PrepParams& p, int b) {
   for (int c = lane; c < nv; c += 32) out[c] = bf16x8_to_f16x8(__ldg(row + c), fa, fb);
 }
 
-__global__ void __launch_bounds__(256, 2) ffn_prep_kernel(const PrepParams p) {
+// Register budgets: rows held in registers (kRegVec 16-byte vectors a lane)
+// take 2 CTAs an SM at 12 vectors, 3 at 8; rows read twice (kRegVec = 0)
+// take 5.  More CTAs keep more of the permuted-row writes of prefill-sized
+// batches in flight.
+template <int kRegVec>
+__global__ void __launch_bounds__(256, kRegVec == 0 ? 5 : kRegVec <= 8 ? 3 : 2) ffn_prep_kernel(const PrepParams p) {
   pdl_enter();
   if (int(blockIdx.x) < p.nsched) prep_schedule(p, blockIdx.x);
-  else prep_rows(p, blockIdx.x - p.nsched);
+  else prep_rows<kRegVec>(p, blockIdx.x - p.nsched);
 }
 
 }  // namespace ftmoe

@@ -59,6 +59,9 @@ static int choose_splits(double units_est, int nkw, int num_sms, double split_co
 constexpr int kPreBN1 = 96, kPreWS1 = 3, kPreBS1 = 4, kPreAS1 = 2, kPreDB1 = 2, kPreKC1 = 64, kPreAM1 = 0;
 constexpr int kPreBN1S = 128, kPreWS1S = 2, kPreBS1S = 3, kPreAS1S = 3, kPreDB1S = 2, kPreKC1S = 64, kPreAM1S = 1;
 constexpr double kGateUpSmemRows = 192.0;
+// Token rows of up to 2048 values: converted from registers (8 vectors a lane)
+// or read twice (0); see ffn_prep_kernel.
+constexpr int kPrepVecSmallH = 8;
 constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 3, kPreAS2 = 2, kPreDB2 = 2, kPreKC2 = 128, kPreAM2 = 0;
 
 // Decode split-K: the largest divisor of the K-stage count that keeps the
@@ -301,7 +304,8 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
     pp.x_perm = reinterpret_cast<uint4*>(x16);
     pp.rowscale = rowscale;
     ProfileScope prof(FT_KERNEL_PREP, s);
-    err = launch_pdl(ffn_prep_kernel, dim3(pp.nsched + (T * k + 7) / 8), dim3(256), 0, s, pp);
+    err = launch_pdl(H <= 2048 ? ffn_prep_kernel<kPrepVecSmallH> : ffn_prep_kernel<12>,
+                     dim3(pp.nsched + (T * k + 7) / 8), dim3(256), 0, s, pp);
   }
   if (err != cudaSuccess) return err;
 
