@@ -64,20 +64,29 @@ constexpr double kGateUpSmemRows = 192.0;
 constexpr int kPrepVecSmallH = 8;
 constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 3, kPreAS2 = 2, kPreDB2 = 2, kPreKC2 = 128, kPreAM2 = 0;
 
-// Decode split-K: the largest divisor of the K-stage count that keeps the
-// units within one wave of the SMs (1 when there are more units than SMs).
-// At a few tokens the kernel is latency-bound: a second wave of units, and
-// each extra split's partial-sum exchange, lengthen the chain from the first
-// weight stage to the last output more than the idle SMs of one wave cost.
-// (Measured on a B200: decode_T1 33.7 vs 36.2 us per layer against the
-// smallest split count that fills every SM; wide_decode_T1 41.8 vs 45.3 us.)
+// Decode split-K.  With at least as many units as SMs: none (the queue keeps
+// every SM busy).  With fewer: the split that minimises the stages on the
+// busiest CTA -- ceil(units * s / SMs) units of sps = ceil(nkw / s) stages --
+// the fewest splits among equals.  A split need not divide the stage count:
+// the last one takes what is left (never nothing, as s = ceil(nkw / sps)).
+// At a few tokens the kernel is latency-bound, and each extra split's
+// partial-sum exchange lengthens the chain from the first weight stage to
+// the last output, so a second wave of units is worth it only where it
+// shortens that chain.  (Measured on a B200: the 48-layer wide_decode_T1
+// sweep 40.4 vs 41.0 us per layer, slots512_T1 33.9 vs 34.9 us, against the
+// largest split count that divides the stages and keeps one wave.)
 static int decode_splits(double units_est, int nkw, int num_sms, int* sps_out) {
-  int best = 1;
-  for (int s = 1; s <= std::min(nkw, 16); ++s) {
-    if (nkw % s) continue;
-    if (units_est * s <= num_sms) best = s;
+  int best = 1, best_sps = nkw;
+  if (units_est < num_sms) {
+    double best_cost = 1e30;
+    for (int sps = nkw; sps >= 1; --sps) {
+      const int s = (nkw + sps - 1) / sps;
+      if (s > 16) break;
+      const double cost = ceil(units_est * s / num_sms - 1e-9) * sps;
+      if (cost < best_cost - 1e-9) { best_cost = cost; best = s; best_sps = sps; }
+    }
   }
-  *sps_out = nkw / best;
+  *sps_out = best_sps;
   return best;
 }
 
