@@ -139,9 +139,19 @@ __device__ __forceinline__ DecUnit decode_unit(const DecodeParams& p, int q, int
 // of the same features; warp w takes features 8w .. 8w+7 -- their gate rows
 // as A rows g and their up rows as A rows g + 8 -- so each thread ends up
 // with both halves of its SwiGLUs.  Down stages: rows 16w .. 16w+15.
-__device__ __forceinline__ int dec_row_lo(int gemm, int w, int g) { return gemm ? 16 * w + g : 8 * w + g; }
+//
+// Inside each group of 8 rows, A row g is row dec_sub(g) = g/2 + 4 (g % 2):
+// the two quads that share a 16-byte load's 8-lane phase (g = 2j, 2j + 1)
+// then read rows whose 128-byte swizzle phases differ in bit 2, so their
+// eight 16-byte code chunks fall in eight different bank groups (with rows
+// g and g + 1 both quads' chunks landed in the same four).  The outputs
+// follow the same map.
+__device__ __forceinline__ int dec_sub(int g) { return (g >> 1) | ((g & 1) << 2); }
+__device__ __forceinline__ int dec_row_lo(int gemm, int w, int g) {
+  return gemm ? 16 * w + dec_sub(g) : 8 * w + dec_sub(g);
+}
 __device__ __forceinline__ int dec_row_hi(int gemm, int w, int g) {
-  return gemm ? 16 * w + 8 + g : kDecFeat1 + 8 * w + g;
+  return gemm ? 16 * w + 8 + dec_sub(g) : kDecFeat1 + 8 * w + dec_sub(g);
 }
 
 // One 256-K stage for this warp: its 16 rows x 256 K x NT token tiles of 8.
@@ -242,7 +252,7 @@ __device__ __forceinline__ bool dec_epilogue(const DecodeParams& p, const DecUni
     }
   }
   if (d.gemm == 0) {
-    const int f = d.mt * kDecFeat1 + 8 * w + g;
+    const int f = d.mt * kDecFeat1 + 8 * w + dec_sub(g);   // the feature of rows r_lo (gate) and r_hi (up)
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -254,7 +264,7 @@ __device__ __forceinline__ bool dec_epilogue(const DecodeParams& p, const DecUni
         }
       }
   } else {
-    const int f = d.mt * kDecRows + 16 * w + g;
+    const int f = d.mt * kDecRows + 16 * w + dec_sub(g);   // row r_lo; r_hi is f + 8
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
