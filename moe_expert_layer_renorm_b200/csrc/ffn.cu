@@ -360,7 +360,7 @@ ffn_gemm_kernel(const FfnParams p, const __grid_constant__ CUtensorMap tm_codes0
     // flag) in the issuing thread leaves the tensor pipe idle for a few
     // hundred cycles even when the operands are already in place.  Warp 3
     // does the waiting; the two warps meet at a named barrier once per chunk,
-    // with warp 3 one chunk ahead, and warp 3 leaves its verdict in
+    // with warp 3 one chunk ahead, and warp 3 leaves its go or stop decision in
     // handoff[q & 1] before it arrives.  Both warps run the same chunk
     // sequence and leave at the same chunk, so every barrier phase completes.
     uint32_t q = 0, di = 0;
