@@ -14,6 +14,7 @@ struct GemmShape { int bn, splits, sps, ws, bs, as, db; };
 struct FfnPlan {
   bool decode;
   bool gu_smem;        // gate/up GEMM in the large-group shape (A in shared memory)
+  bool small;          // both GEMMs in the small-group shape (64-row token tiles, four A slots)
   GemmShape g1, g2;
   int mt1, mt2, nkw1, nkw2, nkc1, nkc2;
   long long max_tiles1, max_tiles2;
@@ -63,6 +64,16 @@ constexpr double kGateUpSmemRows = 192.0;
 // or read twice (0); see ffn_prep_kernel.
 constexpr int kPrepVecSmallH = 8;
 constexpr int kPreBN2 = 192, kPreWS2 = 3, kPreBS2 = 3, kPreAS2 = 2, kPreDB2 = 2, kPreKC2 = 128, kPreAM2 = 0;
+//   both GEMMs, small groups (mean < kSmallGroupRows rows per active expert):
+//     64-row token tiles, which leave tensor memory for four A slots (gate/up:
+//     2 x 2 x 64 accumulator columns + 4 x 2 x 32; down: 2 x 64 + 4 x 64).
+//     With a few dozen rows per group each chunk's MMAs are short, and the
+//     A slot's round trip (dequantise -> MMA -> release) sets the pace; two
+//     slots more keep twice as many chunks in flight.
+constexpr int kPreBN1T = 64, kPreWS1T = 3, kPreBS1T = 4, kPreAS1T = 4, kPreDB1T = 2, kPreKC1T = 64, kPreAM1T = 0;
+constexpr int kPreBN2T = 64, kPreWS2T = 3, kPreBS2T = 4, kPreAS2T = 4, kPreDB2T = 2, kPreKC2T = 128, kPreAM2T = 0;
+constexpr double kSmallGroupRows = 48.0;
+static_assert(kPreKC1T == kPreKC1 && kPreKC1S == kPreKC1 && kPreKC2T == kPreKC2, "one chunk size per GEMM");
 
 // Decode split-K.  With at least as many units as SMs: none (the queue keeps
 // every SM busy).  With fewer: the split that minimises the stages on the
@@ -114,9 +125,12 @@ static FfnPlan plan_ffn(int T, int H, int I, int E, int k, int num_sms) {
     pl.g2 = {kDecBN, 1, 0, 4, 0, 0, 0};
   } else {
     pl.gu_smem = mean_rows >= kGateUpSmemRows;
+    pl.small = mean_rows < kSmallGroupRows;
     pl.g1 = pl.gu_smem ? GemmShape{kPreBN1S, 1, 0, kPreWS1S, kPreBS1S, kPreAS1S, kPreDB1S}
+          : pl.small   ? GemmShape{kPreBN1T, 1, 0, kPreWS1T, kPreBS1T, kPreAS1T, kPreDB1T}
                        : GemmShape{kPreBN1, 1, 0, kPreWS1, kPreBS1, kPreAS1, kPreDB1};
-    pl.g2 = {kPreBN2, 1, 0, kPreWS2, kPreBS2, kPreAS2, kPreDB2};
+    pl.g2 = pl.small ? GemmShape{kPreBN2T, 1, 0, kPreWS2T, kPreBS2T, kPreAS2T, kPreDB2T}
+                     : GemmShape{kPreBN2, 1, 0, kPreWS2, kPreBS2, kPreAS2, kPreDB2};
   }
   const double tiles_per_expert1 = std::max(1.0, ceil(mean_rows / pl.g1.bn));
   const double tiles_per_expert2 = std::max(1.0, ceil(mean_rows / pl.g2.bn));
@@ -320,7 +334,7 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
 
   CUtensorMap tm_x, tm_h;
   if (!make_act_map(x16, T * k, H, pl.decode ? kDecBN : pl.g1.bn, &tm_x) ||
-      !make_act_map(h, T * k, I, pl.decode ? kDecBN : kPreBN2, &tm_h)) {
+      !make_act_map(h, T * k, I, pl.decode ? kDecBN : pl.g2.bn, &tm_h)) {
     *why = "cuTensorMapEncodeTiled failed for the activations";
     return cudaErrorInvalidValue;
   }
@@ -381,10 +395,16 @@ static cudaError_t launch_ffn(const void* x, int T, int H, int I, int E, int k, 
     if (pl.gu_smem)
       err = mx ? launch_gemm<2, kPreBN1S, kPreWS1S, kPreBS1S, kPreAS1S, kPreDB1S, kPreKC1S, FT_SCALE_MXFP4, kPreAM1S>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s)
                : launch_gemm<2, kPreBN1S, kPreWS1S, kPreBS1S, kPreAS1S, kPreDB1S, kPreKC1S, FT_SCALE_NVFP4, kPreAM1S>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
+    else if (pl.small)
+      err = mx ? launch_gemm<2, kPreBN1T, kPreWS1T, kPreBS1T, kPreAS1T, kPreDB1T, kPreKC1T, FT_SCALE_MXFP4, kPreAM1T>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s)
+               : launch_gemm<2, kPreBN1T, kPreWS1T, kPreBS1T, kPreAS1T, kPreDB1T, kPreKC1T, FT_SCALE_NVFP4, kPreAM1T>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
     else
       err = mx ? launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1, FT_SCALE_MXFP4, kPreAM1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s)
                : launch_gemm<2, kPreBN1, kPreWS1, kPreBS1, kPreAS1, kPreDB1, kPreKC1, FT_SCALE_NVFP4, kPreAM1>(p1, grid1, tmc[0], tms[0], tmc[1], tms[1], tm_x, s);
-    if (err == cudaSuccess)
+    if (err == cudaSuccess && pl.small)
+      err = mx ? launch_gemm<1, kPreBN2T, kPreWS2T, kPreBS2T, kPreAS2T, kPreDB2T, kPreKC2T, FT_SCALE_MXFP4, kPreAM2T>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s)
+               : launch_gemm<1, kPreBN2T, kPreWS2T, kPreBS2T, kPreAS2T, kPreDB2T, kPreKC2T, FT_SCALE_NVFP4, kPreAM2T>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
+    else if (err == cudaSuccess)
       err = mx ? launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2, FT_SCALE_MXFP4, kPreAM2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s)
                : launch_gemm<1, kPreBN2, kPreWS2, kPreBS2, kPreAS2, kPreDB2, kPreKC2, FT_SCALE_NVFP4, kPreAM2>(p2, grid2, tmc[2], tms[2], tmc[2], tms[2], tm_h, s);
   }

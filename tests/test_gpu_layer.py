@@ -29,13 +29,27 @@ def test_layer_full_parity(cuda_device, name):
 
 
 @pytest.mark.parametrize("H,I,E,k,T", [(320, 448, 8, 2, 40), (256, 256, 4, 4, 100), (576, 320, 16, 3, 333),
-                                         (320, 448, 4, 2, 600), (576, 2880, 3, 2, 700)])
+                                         (320, 448, 4, 2, 600), (576, 2880, 3, 2, 700),
+                                         (320, 448, 32, 2, 400), (576, 320, 64, 4, 600)])
 def test_ragged_shapes(cuda_device, H, I, E, k, T):
     # K not a multiple of 256, output features not a multiple of 128, groups spanning several tiles; the
-    # last two have hundreds of rows per expert (the gate/up GEMM's large-group shape)
+    # 4th and 5th have hundreds of rows per expert (the gate/up GEMM's large-group shape), the last two a few
+    # dozen (both GEMMs' small-group shape: 64-row token tiles)
     w = inputs.custom_workload(W["tiny"], H=H, I=I, E=E, k=k, T=T, seed=4242 + H)
     run = G.run_gpu(w)
     G.check_routing(run, w.k)
+    G.check_output(run, w.k)
+
+
+def test_small_groups_skewed(cuda_device):
+    # a few dozen rows per expert on average (the small-group shape) with Zipf-skewed routing, so that some
+    # groups take several 64-row tiles and others none
+    w = inputs.custom_workload(W["tiny"], H=256, I=512, E=64, k=2, T=700, zipf_s=1.1, seed=4711)
+    run = G.run_gpu(w)
+    G.check_routing(run, w.k)
+    counts = np.diff(run.layer.offsets.cpu().numpy())
+    assert counts.max() > 128 and counts.min() < 8
+    assert 16 < w.T * w.k / max(1, int((counts > 0).sum())) < 48
     G.check_output(run, w.k)
 
 
